@@ -1,0 +1,527 @@
+#!/usr/bin/env python
+"""Benchmark of the blockwise-FP8 training-linear hot path on B200.
+
+One step = the whole hot path over the linear stack of one 28-layer
+Qwen3-1.7B-shaped training step at M = 16384 tokens (4 x 4096): for every
+layer and each of its four linears (QKV 2048->4096, O 2048->2048, gate/up
+2048->12288, down 6144->2048):
+  1. 128x128 block quantisation of W (codes + transposed codes + scales)
+  2. row-wise + column-wise 1x128 / 128x1 quantisation of X (one pass)
+  3. fprop  Y  = X W^T
+  4. row-wise + column-wise quantisation of dY (one pass)
+  5. dgrad  dX = dY W
+  6. wgrad  dW = dY^T X
+= 672 kernel launches, 138.5 TFLOP of GEMM work per step.
+
+Inputs are seeded synthetic tensors (synthetic/): X ~ N(0,1) with 0.1% x50
+outliers, W ~ N(0,0.02), dY ~ N(0,1e-3) with 0.1% x100 outliers. Every layer
+reuses its linear's input buffers; between two uses of a buffer the step
+streams more than 1 GB through HBM (8x the 126 MB L2), so every launch reads
+cold data ("inputs larger than L2").
+
+Metric: GEMM TFLOP/s of the whole step (quantiser time included in the step
+time). The JSON line also carries per-kernel achieved TFLOP/s or GB/s (CUDA
+events around every launch of the timed region), the roofline of the
+dominant kernel, the clocks seen during the timed region, an end-to-end
+number with host<->device copies in the timed region, and the CPU oracle on
+a bounded sample of the same workload.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+WORKLOAD = "stack28_m16384"
+LAYERS = 28
+TOKENS = 16384
+METRIC = ("blockwise-FP8 GEMM TFLOP/s (fwd/dgrad/wgrad) & % FP8 peak; "
+          "quantize GB/s % HBM")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
+                  "bf16_tflops_sustained": 1400.0}
+FP8_OVER_BF16 = 2.0   # nominal dense FP8 / BF16 tensor throughput (4.5 / 2.25)
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def kinds():
+    from synthetic import LINEARS
+    return [(kind, LINEARS[kind][0], LINEARS[kind][1])
+            for kind in ("qkv", "o", "gate_up", "down")]
+
+
+def step_gemm_flops():
+    return LAYERS * 3 * sum(2 * TOKENS * n * k for _, k, n in kinds())
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            d = json.load(fh)
+        return {"hbm_gbs": float(d["hbm_gbs"]),
+                "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d["bf16_tflops_sustained"]),
+                "source": "measured"}
+    except Exception:
+        d = dict(FALLBACK_PEAKS)
+        d["source"] = "fallback"
+        return d
+
+
+# --------------------------------------------------------------------------
+# CPU oracle on a bounded sample (the reference arm, and the cpu_baseline)
+# --------------------------------------------------------------------------
+
+class OracleSample:
+    """The four linears of one layer at a reduced token count M' (instead of
+    16384), plus quantisation of the same fraction of each weight; every GEMM
+    and quantiser of the step scales linearly with M', so the sample's
+    throughput stands for the step's."""
+
+    def __init__(self, tokens):
+        import oracle
+        import synthetic as S
+        self.oracle = oracle
+        self.tokens = tokens
+        self.threads = oracle.default_threads()
+        self.items = []
+        for kind, k, n in kinds():
+            lin = S.Linear(kind, tokens, k, n, ("fprop", "dgrad", "wgrad"))
+            w = S.draw_w(lin)
+            qw, sw, _ = oracle.quantize_weight_block(w, want_transposed=False)
+            wrows = max(16, (n * tokens // TOKENS) // 16 * 16)
+            self.items.append(dict(x=S.draw_x(lin), dy=S.draw_dy(lin),
+                                   w_slab=np.ascontiguousarray(w[:wrows]),
+                                   qw=qw, sw=sw, m=tokens, n=n, k=k))
+        self.flops = sum(3 * 2 * it["m"] * it["n"] * it["k"]
+                         for it in self.items)
+
+    def run(self):
+        o = self.oracle
+        nt = self.threads
+        for it in self.items:
+            o.quantize_weight_block(it["w_slab"], want_transposed=True)
+            qx, sx = o.quantize_rowwise(it["x"])
+            qx_t, sx_t = o.quantize_colwise(it["x"])
+            o.gemm_fprop(qx, sx, it["qw"], it["sw"], nthreads=nt)
+            qdy, sdy = o.quantize_rowwise(it["dy"])
+            qdy_t, sdy_t = o.quantize_colwise(it["dy"])
+            o.gemm_dgrad(qdy, sdy, it["qw"], it["sw"], nthreads=nt)
+            o.gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t, nthreads=nt)
+
+    def describe(self):
+        return ("the 4 linears of one layer (QKV, O, gate/up, down) at %d "
+                "tokens instead of %d (1/%d of every GEMM and activation "
+                "quantisation) plus 1/%d of each weight's block quantisation; "
+                "fp64 oracle GEMMs on %d threads"
+                % (self.tokens, TOKENS, TOKENS // self.tokens,
+                   TOKENS // self.tokens, self.threads))
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    sample = OracleSample(tokens=64)
+    for _ in range(args.warmup):
+        sample.run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        sample.run()
+    dt = (time.perf_counter() - t0) / args.steps
+    value = sample.flops / dt / 1e12
+    line = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": args.gpus,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": dt * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "layers": LAYERS, "tokens": TOKENS,
+                   "sample_tokens": sample.tokens},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s",
+                         "cores": sample.threads, "kind": "oracle",
+                         "sample": sample.describe()},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# --------------------------------------------------------------------------
+# GPU arm
+# --------------------------------------------------------------------------
+
+class LinearBuffers:
+    """Device buffers of one linear kind (inputs + every intermediate)."""
+
+    def __init__(self, kind, k, n, device):
+        import torch
+        import synthetic as S
+        self.kind, self.k, self.n = kind, k, n
+        m = TOKENS
+        lin = S.Linear(kind, m, k, n, ("fprop", "dgrad", "wgrad"))
+        self.host_x = S.draw_x(lin)
+        self.host_w = S.draw_w(lin)
+        self.host_dy = S.draw_dy(lin)
+
+        def dev_bf16(a):
+            t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+            return t.to(device)
+
+        def e(shape, dt):
+            return torch.empty(shape, dtype=dt, device=device)
+
+        u8, f32, bf = torch.uint8, torch.float32, torch.bfloat16
+        self.x, self.w, self.dy = (dev_bf16(self.host_x),
+                                   dev_bf16(self.host_w),
+                                   dev_bf16(self.host_dy))
+        cd = lambda a: (a + 127) // 128  # noqa: E731
+        self.qw, self.sw, self.qw_t = e((n, k), u8), e((cd(n), cd(k)), f32), \
+            e((k, n), u8)
+        self.qx, self.sx = e((m, k), u8), e((cd(k), m), f32)
+        self.qx_t, self.sx_t = e((k, m), u8), e((cd(m), k), f32)
+        self.qdy, self.sdy = e((m, n), u8), e((cd(n), m), f32)
+        self.qdy_t, self.sdy_t = e((n, m), u8), e((cd(m), n), f32)
+        self.y, self.dx, self.dw = e((m, n), bf), e((m, k), bf), e((n, k), bf)
+
+    def ops(self, o, stream):
+        """[(kernel kind, algorithmic units, callable)] of this linear."""
+        m, k, n = TOKENS, self.k, self.n
+        cd = lambda a: (a + 127) // 128  # noqa: E731
+        wq_bytes = n * k * 2 + 2 * n * k + 4 * cd(n) * cd(k)
+        xq_bytes = m * k * 2 + 2 * m * k + 4 * (m * cd(k) + cd(m) * k)
+        dyq_bytes = m * n * 2 + 2 * m * n + 4 * (m * cd(n) + cd(m) * n)
+        f = 2 * m * n * k
+        return [
+            ("quant_weight_block", wq_bytes,
+             lambda: o.fp8bw_quantize_weight_block(self.w, self.qw, self.sw,
+                                                   self.qw_t, stream)),
+            ("quant_rowcol", xq_bytes,
+             lambda: o.fp8bw_quantize_colwise(self.x, self.qx_t, self.sx_t,
+                                              self.qx, self.sx, stream)),
+            ("gemm_block_scaled", f,
+             lambda: o.fp8bw_gemm_fprop(self.qx, self.sx, self.qw, self.sw,
+                                        self.y, stream)),
+            ("quant_rowcol", dyq_bytes,
+             lambda: o.fp8bw_quantize_colwise(self.dy, self.qdy_t,
+                                              self.sdy_t, self.qdy,
+                                              self.sdy, stream)),
+            ("gemm_block_scaled", f,
+             lambda: o.fp8bw_gemm_dgrad(self.qdy, self.sdy, self.qw_t, 1,
+                                        self.sw, self.dx, stream)),
+            ("gemm_vector_scaled", f,
+             lambda: o.fp8bw_gemm_wgrad(self.qdy_t, self.sdy_t, self.qx_t,
+                                        self.sx_t, self.dw, stream)),
+        ]
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200", "-i",
+                 gpu_id], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        mhz, maxes, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                maxes.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not mhz:
+            return None
+        return {"sm_mhz": statistics.median(mhz),
+                "sm_max_mhz": max(maxes) if maxes else None,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+def gpu_uuid(torch, dev):
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(dev)
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", device_id=dev,
+                                timeout=datetime.timedelta(seconds=300))
+
+    from blockwise_fp8_linear_fp8bw_b200 import ops as o
+
+    stream = torch.cuda.Stream(device=dev)
+    bufs = [LinearBuffers(kind, k, n, dev) for kind, k, n in kinds()]
+    step_ops = []
+    for _layer in range(LAYERS):
+        for b in bufs:
+            step_ops.extend(b.ops(o, stream))
+    flops = step_gemm_flops()
+    assert flops == sum(u for kk, u, _ in step_ops if kk.startswith("gemm"))
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    def run_step(events=None):
+        if events is None:
+            for _, _, fn in step_ops:
+                fn()
+        else:
+            for (_, _, fn), (e0, e1) in zip(step_ops, events):
+                e0.record(stream)
+                fn()
+                e1.record(stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            run_step()
+    torch.cuda.synchronize()
+    o.fp8bw_check_device_error(stream)
+
+    events = [[(torch.cuda.Event(enable_timing=True),
+                torch.cuda.Event(enable_timing=True)) for _ in step_ops]
+              for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(gpu_uuid(torch, dev))
+    time.sleep(0.6)
+    barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        t_start.record(stream)
+        for s in range(args.steps):
+            run_step(events[s])
+        t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    o.fp8bw_check_device_error(stream)
+    ms = t_start.elapsed_time(t_end) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # per-kernel durations inside the timed region
+    per_kind = {}
+    for s in range(args.steps):
+        for (kk, units, _), (e0, e1) in zip(step_ops, events[s]):
+            d = per_kind.setdefault(kk, {"ms": 0.0, "units": 0, "launches": 0})
+            d["ms"] += e0.elapsed_time(e1)
+            d["units"] += units
+            d["launches"] += 1
+
+    # ---------------------------------------------------------- end to end
+    e2e = None
+    if not args.no_e2e:
+        pinned = []
+        for b in bufs:
+            hx = torch.from_numpy(b.host_x.view(np.int16)).view(
+                torch.bfloat16).pin_memory()
+            hw = torch.from_numpy(b.host_w.view(np.int16)).view(
+                torch.bfloat16).pin_memory()
+            hdy = torch.from_numpy(b.host_dy.view(np.int16)).view(
+                torch.bfloat16).pin_memory()
+            hdw = torch.empty(b.dw.shape, dtype=torch.bfloat16).pin_memory()
+            pinned.append((hx, hw, hdy, hdw))
+        h2d = LAYERS * sum(p[0].numel() * 2 + p[1].numel() * 2 +
+                           p[2].numel() * 2 for p in pinned)
+        d2h = LAYERS * sum(p[3].numel() * 2 for p in pinned)
+
+        def e2e_step():
+            for _layer in range(LAYERS):
+                for b, (hx, hw, hdy, hdw) in zip(bufs, pinned):
+                    b.x.copy_(hx, non_blocking=True)
+                    b.w.copy_(hw, non_blocking=True)
+                    b.dy.copy_(hdy, non_blocking=True)
+                    for _, _, fn in b.ops(o, stream):
+                        fn()
+                    hdw.copy_(b.dw, non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                e2e_step()
+        torch.cuda.synchronize()
+        e_s = torch.cuda.Event(enable_timing=True)
+        e_e = torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            e_s.record(stream)
+            for _ in range(args.steps):
+                e2e_step()
+            e_e.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        o.fp8bw_check_device_error(stream)
+        e2e_ms = e_s.elapsed_time(e_e) / args.steps
+        if world > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * flops / (e2e_ms * 1e-3) / 1e12,
+               "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks = load_peaks()
+    fp8_sustained = peaks["bf16_tflops_sustained"] * FP8_OVER_BF16
+    breakdown = {}
+    for kk, d in sorted(per_kind.items()):
+        avg_ms = d["ms"] / d["launches"]
+        if kk.startswith("gemm"):
+            ach = d["units"] / (d["ms"] * 1e-3) / 1e12
+            breakdown[kk] = {"achieved": ach, "unit": "TFLOP/s",
+                             "frac_of_fp8_peak": ach / fp8_sustained,
+                             "share": d["ms"] / (ms * args.steps),
+                             "launches_per_step": d["launches"] // args.steps,
+                             "avg_launch_ms": avg_ms}
+        else:
+            ach = d["units"] / (d["ms"] * 1e-3) / 1e9
+            breakdown[kk] = {"achieved": ach, "unit": "GB/s",
+                             "frac_of_hbm": ach / peaks["hbm_gbs"],
+                             "share": d["ms"] / (ms * args.steps),
+                             "launches_per_step": d["launches"] // args.steps,
+                             "avg_launch_ms": avg_ms}
+    dom = max(per_kind.items(), key=lambda kv: kv[1]["ms"])
+    dk, dd = dom
+    if dk.startswith("gemm"):
+        ach = dd["units"] / (dd["ms"] * 1e-3) / 1e12
+        roofline = {"kernel": dk, "bound": "tensor", "achieved": ach,
+                    "peak": fp8_sustained, "unit": "TFLOP/s",
+                    "frac": ach / fp8_sustained, "traffic": None,
+                    "peak_note": "%s sustained bf16 x %.0f (nominal FP8/BF16)"
+                    % (peaks["source"], FP8_OVER_BF16)}
+    else:
+        ach = dd["units"] / (dd["ms"] * 1e-3) / 1e9
+        roofline = {"kernel": dk, "bound": "hbm", "achieved": ach,
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": ach / peaks["hbm_gbs"], "traffic": None,
+                    "peak_note": "%s copy bandwidth" % peaks["source"]}
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        sample = OracleSample(tokens=256)
+        t0 = time.perf_counter()
+        sample.run()
+        dt = time.perf_counter() - t0
+        cpu = {"value": sample.flops / dt / 1e12, "unit": "TFLOP/s",
+               "cores": sample.threads, "kind": "oracle",
+               "sample": sample.describe(), "seconds": dt}
+
+    value = world * flops / (ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e4m3",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "layers": LAYERS, "tokens": TOKENS,
+                   "linears": {kd: [k, n] for kd, k, n in kinds()},
+                   "gemm_tflop_per_step": flops / 1e12,
+                   "l2": "inputs larger than L2 (>1 GB streamed between "
+                         "reuses of any buffer)",
+                   "parallelism": "replicas" if world > 1 else "single"},
+        "gpu_launches": len(step_ops) * args.steps,
+        "roofline": roofline,
+        "breakdown": breakdown,
+        "clocks": clk,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "peaks": {"hbm_gbs": peaks["hbm_gbs"],
+                  "fp8_tflops_sustained": fp8_sustained,
+                  "source": peaks["source"]},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

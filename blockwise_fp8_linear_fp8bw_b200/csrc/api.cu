@@ -1,0 +1,374 @@
+// api.cu -- the library's C ABI (declared in include/fp8bw.h): argument
+// validation, TMA descriptor encoding and kernel launches. The whole library
+// is this one translation unit (the kernels come in as headers) so that the
+// device error record is a single symbol without relocatable device code.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "gemm.cuh"
+#include "quant.cuh"
+
+namespace fp8bw {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  int checked = 0;      // 0 = unknown, 1 = sm_100, -1 = other
+  int sm_count = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+int current_device_info(DeviceInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return FP8BW_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (d.checked == 0) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return FP8BW_ERR_DEVICE;
+    d.checked = (major == 10 && minor == 0) ? 1 : -1;
+    d.sm_count = sms;
+  }
+  if (d.checked != 1) return FP8BW_ERR_DEVICE;
+  *out = d;
+  return FP8BW_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool dim_ok(int64_t d) { return d >= 0 && (d % 16) == 0 && d <= (int64_t(1) << 30); }
+
+struct Range {
+  uintptr_t lo, hi;  // [lo, hi)
+};
+Range range_of(const void* p, int64_t bytes) {
+  uintptr_t b = reinterpret_cast<uintptr_t>(p);
+  return Range{b, b + static_cast<uintptr_t>(bytes > 0 ? bytes : 0)};
+}
+bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi && a.lo != a.hi && b.lo != b.hi; }
+
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// A pointer may be NULL only when its buffer holds no element.
+bool missing(const void* p, int64_t bytes) { return p == nullptr && bytes > 0; }
+
+// --------------------------------------------------------------- TMA encode
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int get_encode(PFN_cuTensorMapEncodeTiled_v12000* fn) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_encode == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || p == nullptr)
+      return FP8BW_ERR_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  *fn = g_encode;
+  return FP8BW_OK;
+}
+
+// 2-D uint8 tensor [outer, inner] (row pitch = inner bytes), box [box_outer,
+// 128 bytes], 128-byte swizzle; out-of-range elements read as zero.
+int encode_u8_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                 uint32_t box_outer) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  int st = get_encode(&enc);
+  if (st != FP8BW_OK) return st;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner};
+  cuuint32_t box[2] = {128u, box_outer};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FP8BW_OK : FP8BW_ERR_CUDA;
+}
+
+// --------------------------------------------------------------- GEMM launch
+struct GemmProblem {
+  const uint8_t* a;  // [mo][kc]
+  const uint8_t* b;  // K-major: [no][kc]; MN-major: [kc][no]
+  bool b_mn;
+  bool vec_b;
+  int64_t mo, no, kc;
+  const float* sa;
+  const float* sb;
+  int64_t sbj, sbc;
+  uint16_t* out;
+};
+
+template <int BN, bool VEC_B, bool B_MN>
+int launch_gemm_t(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t stream) {
+  using L = gemm::Layout<BN, VEC_B>;
+  auto kernel = gemm::blockwise_gemm_kernel<BN, VEC_B, B_MN>;
+  static std::once_flag once;
+  static int prep_status = FP8BW_OK;
+  std::call_once(once, [&]() {
+    cudaFuncAttributes attr;
+    if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess) {
+      prep_status = FP8BW_ERR_LAUNCH;
+      return;
+    }
+    // setmaxnreg redistributes exactly the registers the CTA was launched
+    // with; a smaller launch allocation would make the increase wait forever.
+    if (attr.numRegs < gemm::kLaunchRegs) {
+      prep_status = FP8BW_ERR_LAUNCH;
+      return;
+    }
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             L::kAlloc) != cudaSuccess)
+      prep_status = FP8BW_ERR_LAUNCH;
+  });
+  if (prep_status != FP8BW_OK) return prep_status;
+
+  CUtensorMap tm_a, tm_b;
+  int st = encode_u8_2d(&tm_a, p.a, static_cast<uint64_t>(p.kc), static_cast<uint64_t>(p.mo),
+                        gemm::BM);
+  if (st != FP8BW_OK) return st;
+  if (B_MN)
+    st = encode_u8_2d(&tm_b, p.b, static_cast<uint64_t>(p.no), static_cast<uint64_t>(p.kc), 128);
+  else
+    st = encode_u8_2d(&tm_b, p.b, static_cast<uint64_t>(p.kc), static_cast<uint64_t>(p.no), BN);
+  if (st != FP8BW_OK) return st;
+
+  gemm::Args g;
+  g.mo = static_cast<int>(p.mo);
+  g.no = static_cast<int>(p.no);
+  g.kc = static_cast<int>(p.kc);
+  g.tiles_m = static_cast<int>(cdiv(p.mo, gemm::BM));
+  g.tiles_n = static_cast<int>(cdiv(p.no, BN));
+  g.chunks = static_cast<int>(cdiv(p.kc, gemm::BK));
+  g.sa = p.sa;
+  g.sb = p.sb;
+  g.sbj = p.sbj;
+  g.sbc = p.sbc;
+  g.nblk = static_cast<int>(cdiv(p.no, 128));
+  g.out = p.out;
+  const int tiles = g.tiles_m * g.tiles_n;
+  const int grid = std::min(tiles, dev.sm_count);
+  kernel<<<grid, gemm::kThreads, L::kAlloc, stream>>>(tm_a, tm_b, g);
+  return cudaGetLastError() == cudaSuccess ? FP8BW_OK : FP8BW_ERR_LAUNCH;
+}
+
+int run_gemm(const GemmProblem& p, cudaStream_t stream) {
+  DeviceInfo dev;
+  int st = current_device_info(&dev);
+  if (st != FP8BW_OK) return st;
+  if (p.mo == 0 || p.no == 0) return FP8BW_OK;
+  if (p.kc == 0) {
+    return cudaMemsetAsync(p.out, 0, static_cast<size_t>(p.mo * p.no * 2), stream) == cudaSuccess
+               ? FP8BW_OK
+               : FP8BW_ERR_CUDA;
+  }
+  if (p.vec_b) return launch_gemm_t<256, true, false>(p, dev, stream);
+  if (p.b_mn) return launch_gemm_t<256, false, true>(p, dev, stream);
+  return launch_gemm_t<256, false, false>(p, dev, stream);
+}
+
+}  // namespace
+}  // namespace fp8bw
+
+using namespace fp8bw;
+
+extern "C" {
+
+int fp8bw_version(void) { return 100; }
+
+const char* fp8bw_status_string(int status) {
+  switch (status) {
+    case FP8BW_OK: return "ok";
+    case FP8BW_ERR_NULL: return "a required pointer is NULL";
+    case FP8BW_ERR_SHAPE: return "a dimension is negative, not a multiple of 16, or too large";
+    case FP8BW_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case FP8BW_ERR_DEVICE: return "the current CUDA device is not compute capability 10.0 (sm_100)";
+    case FP8BW_ERR_LAUNCH: return "kernel launch failed";
+    case FP8BW_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait expired";
+    case FP8BW_ERR_CUDA: return "a CUDA runtime or driver call failed";
+    case FP8BW_ERR_ALIAS: return "an output buffer overlaps an input buffer";
+    default: return "unknown status";
+  }
+}
+
+int fp8bw_quantize_rowwise(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* q, float* s,
+                           void* stream) {
+  if (!dim_ok(rows) || !dim_ok(cols) || cdiv(rows, 128) > 65535) return FP8BW_ERR_SHAPE;
+  if (missing(x, rows * cols) || missing(q, rows * cols) || missing(s, cdiv(cols, 128) * rows))
+    return FP8BW_ERR_NULL;
+  if (!aligned16(x) || !aligned16(q) || !aligned16(s)) return FP8BW_ERR_ALIGN;
+  const Range rx = range_of(x, rows * cols * 2);
+  if (overlap(rx, range_of(q, rows * cols)) || overlap(rx, range_of(s, cdiv(cols, 128) * rows * 4)))
+    return FP8BW_ERR_ALIAS;
+  DeviceInfo dev;
+  int st = current_device_info(&dev);
+  if (st != FP8BW_OK) return st;
+  if (rows == 0 || cols == 0) return FP8BW_OK;
+  return launch_quantize(kModeRow, x, rows, cols, q, s, nullptr, nullptr, nullptr,
+                         static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? FP8BW_OK
+             : FP8BW_ERR_LAUNCH;
+}
+
+int fp8bw_quantize_colwise(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* q_t,
+                           float* s_t, uint8_t* q_row, float* s_row, void* stream) {
+  if (!dim_ok(rows) || !dim_ok(cols) || cdiv(rows, 128) > 65535) return FP8BW_ERR_SHAPE;
+  if (missing(x, rows * cols) || missing(q_t, rows * cols) || missing(s_t, cdiv(rows, 128) * cols))
+    return FP8BW_ERR_NULL;
+  if (rows * cols > 0 && (q_row == nullptr) != (s_row == nullptr)) return FP8BW_ERR_NULL;
+  if (!aligned16(x) || !aligned16(q_t) || !aligned16(s_t) || !aligned16(q_row) ||
+      !aligned16(s_row))
+    return FP8BW_ERR_ALIGN;
+  const Range rx = range_of(x, rows * cols * 2);
+  if (overlap(rx, range_of(q_t, rows * cols)) ||
+      overlap(rx, range_of(s_t, cdiv(rows, 128) * cols * 4)) ||
+      (q_row && (overlap(rx, range_of(q_row, rows * cols)) ||
+                 overlap(rx, range_of(s_row, cdiv(cols, 128) * rows * 4)))))
+    return FP8BW_ERR_ALIAS;
+  DeviceInfo dev;
+  int st = current_device_info(&dev);
+  if (st != FP8BW_OK) return st;
+  if (rows == 0 || cols == 0) return FP8BW_OK;
+  const int mode = q_row ? kModeRowCol : kModeCol;
+  return launch_quantize(mode, x, rows, cols, q_row, s_row, q_t, s_t, nullptr,
+                         static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? FP8BW_OK
+             : FP8BW_ERR_LAUNCH;
+}
+
+int fp8bw_quantize_weight_block(const uint16_t* w, int64_t n, int64_t k, uint8_t* q, float* s,
+                                uint8_t* q_t, void* stream) {
+  if (!dim_ok(n) || !dim_ok(k) || cdiv(n, 128) > 65535) return FP8BW_ERR_SHAPE;
+  if (missing(w, n * k) || missing(q, n * k) || missing(s, cdiv(n, 128) * cdiv(k, 128)))
+    return FP8BW_ERR_NULL;
+  if (!aligned16(w) || !aligned16(q) || !aligned16(s) || !aligned16(q_t)) return FP8BW_ERR_ALIGN;
+  const Range rw = range_of(w, n * k * 2);
+  if (overlap(rw, range_of(q, n * k)) || overlap(rw, range_of(s, cdiv(n, 128) * cdiv(k, 128) * 4)) ||
+      (q_t && overlap(rw, range_of(q_t, n * k))))
+    return FP8BW_ERR_ALIAS;
+  DeviceInfo dev;
+  int st = current_device_info(&dev);
+  if (st != FP8BW_OK) return st;
+  if (n == 0 || k == 0) return FP8BW_OK;
+  return launch_quantize(kModeBlock, w, n, k, q, nullptr, q_t, nullptr, s,
+                         static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? FP8BW_OK
+             : FP8BW_ERR_LAUNCH;
+}
+
+int fp8bw_gemm_fprop(const uint8_t* qx, const float* sx, const uint8_t* qw, const float* sw,
+                     int64_t m, int64_t n, int64_t k, uint16_t* y, void* stream) {
+  if (!dim_ok(m) || !dim_ok(n) || !dim_ok(k)) return FP8BW_ERR_SHAPE;
+  if (missing(qx, m * k) || missing(sx, cdiv(k, 128) * m) || missing(qw, n * k) ||
+      missing(sw, cdiv(n, 128) * cdiv(k, 128)) || missing(y, m * n))
+    return FP8BW_ERR_NULL;
+  if (!aligned16(qx) || !aligned16(sx) || !aligned16(qw) || !aligned16(sw) || !aligned16(y))
+    return FP8BW_ERR_ALIGN;
+  const Range ry = range_of(y, m * n * 2);
+  if (overlap(ry, range_of(qx, m * k)) || overlap(ry, range_of(sx, cdiv(k, 128) * m * 4)) ||
+      overlap(ry, range_of(qw, n * k)) || overlap(ry, range_of(sw, cdiv(n, 128) * cdiv(k, 128) * 4)))
+    return FP8BW_ERR_ALIAS;
+  GemmProblem p{};
+  p.a = qx;
+  p.b = qw;
+  p.b_mn = false;
+  p.vec_b = false;
+  p.mo = m;
+  p.no = n;
+  p.kc = k;
+  p.sa = sx;
+  p.sb = sw;
+  p.sbj = cdiv(k, 128);  // sW[n/128][c]
+  p.sbc = 1;
+  p.out = y;
+  return run_gemm(p, static_cast<cudaStream_t>(stream));
+}
+
+int fp8bw_gemm_dgrad(const uint8_t* qdy, const float* sdy, const uint8_t* qw,
+                     int qw_is_transposed, const float* sw, int64_t m, int64_t n, int64_t k,
+                     uint16_t* dx, void* stream) {
+  if (!dim_ok(m) || !dim_ok(n) || !dim_ok(k)) return FP8BW_ERR_SHAPE;
+  if (missing(qdy, m * n) || missing(sdy, cdiv(n, 128) * m) || missing(qw, n * k) ||
+      missing(sw, cdiv(n, 128) * cdiv(k, 128)) || missing(dx, m * k))
+    return FP8BW_ERR_NULL;
+  if (!aligned16(qdy) || !aligned16(sdy) || !aligned16(qw) || !aligned16(sw) || !aligned16(dx))
+    return FP8BW_ERR_ALIGN;
+  const Range rd = range_of(dx, m * k * 2);
+  if (overlap(rd, range_of(qdy, m * n)) || overlap(rd, range_of(sdy, cdiv(n, 128) * m * 4)) ||
+      overlap(rd, range_of(qw, n * k)) || overlap(rd, range_of(sw, cdiv(n, 128) * cdiv(k, 128) * 4)))
+    return FP8BW_ERR_ALIAS;
+  GemmProblem p{};
+  p.a = qdy;
+  p.b = qw;
+  p.b_mn = qw_is_transposed == 0;  // qW [n, k]: output columns contiguous
+  p.vec_b = false;
+  p.mo = m;
+  p.no = k;
+  p.kc = n;
+  p.sa = sdy;
+  p.sb = sw;
+  p.sbj = 1;             // sW[c][k/128]
+  p.sbc = cdiv(k, 128);
+  p.out = dx;
+  return run_gemm(p, static_cast<cudaStream_t>(stream));
+}
+
+int fp8bw_gemm_wgrad(const uint8_t* qdy_t, const float* sdy_t, const uint8_t* qx_t,
+                     const float* sx_t, int64_t m, int64_t n, int64_t k, uint16_t* dw,
+                     void* stream) {
+  if (!dim_ok(m) || !dim_ok(n) || !dim_ok(k)) return FP8BW_ERR_SHAPE;
+  if (missing(qdy_t, n * m) || missing(sdy_t, cdiv(m, 128) * n) || missing(qx_t, k * m) ||
+      missing(sx_t, cdiv(m, 128) * k) || missing(dw, n * k))
+    return FP8BW_ERR_NULL;
+  if (!aligned16(qdy_t) || !aligned16(sdy_t) || !aligned16(qx_t) || !aligned16(sx_t) ||
+      !aligned16(dw))
+    return FP8BW_ERR_ALIGN;
+  const Range rd = range_of(dw, n * k * 2);
+  if (overlap(rd, range_of(qdy_t, n * m)) || overlap(rd, range_of(sdy_t, cdiv(m, 128) * n * 4)) ||
+      overlap(rd, range_of(qx_t, k * m)) || overlap(rd, range_of(sx_t, cdiv(m, 128) * k * 4)))
+    return FP8BW_ERR_ALIAS;
+  GemmProblem p{};
+  p.a = qdy_t;
+  p.b = qx_t;
+  p.b_mn = false;
+  p.vec_b = true;
+  p.mo = n;
+  p.no = k;
+  p.kc = m;
+  p.sa = sdy_t;
+  p.sb = sx_t;
+  p.sbj = 0;
+  p.sbc = 0;
+  p.out = dw;
+  return run_gemm(p, static_cast<cudaStream_t>(stream));
+}
+
+int fp8bw_check_device_error(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return FP8BW_ERR_CUDA;
+  uint32_t v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, fp8bw::g_device_error, sizeof v) != cudaSuccess)
+    return FP8BW_ERR_CUDA;
+  if (v != 0u &&
+      cudaMemcpyToSymbol(fp8bw::g_device_error, &zero, sizeof zero) != cudaSuccess)
+    return FP8BW_ERR_CUDA;
+  return v != 0u ? FP8BW_ERR_DEVICE_TIMEOUT : FP8BW_OK;
+}
+
+}  // extern "C"

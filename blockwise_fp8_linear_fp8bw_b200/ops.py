@@ -1,0 +1,202 @@
+"""Python binding of the C ABI: the same entry points, taking torch tensors.
+
+Argument marshalling only (tensor -> device pointer, shape -> int64, the
+current CUDA stream -> cudaStream_t); every step of the computation runs in
+the CUDA library. The `fp8bw_*` functions take pre-allocated outputs; the
+short-named helpers allocate the outputs with torch and call them.
+"""
+import torch
+
+from . import _native
+
+FP8BW_OK = 0
+FP8BW_ERR_NULL = -1
+FP8BW_ERR_SHAPE = -2
+FP8BW_ERR_ALIGN = -3
+FP8BW_ERR_DEVICE = -4
+FP8BW_ERR_LAUNCH = -5
+FP8BW_ERR_DEVICE_TIMEOUT = -6
+FP8BW_ERR_CUDA = -7
+FP8BW_ERR_ALIAS = -8
+
+_lib = _native.load()
+
+
+class Fp8bwError(RuntimeError):
+    def __init__(self, status: int, call: str):
+        self.status = status
+        msg = _lib.fp8bw_status_string(status).decode()
+        super().__init__("%s failed: %s (%d)" % (call, msg, status))
+
+
+def _check(status: int, call: str) -> None:
+    if status != FP8BW_OK:
+        raise Fp8bwError(status, call)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _expect(t, dtype, shape, name):
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape):
+        raise ValueError("%s: expected %s %s, got %s %s" %
+                         (name, dtype, tuple(shape), t.dtype, tuple(t.shape)))
+
+
+def _cdiv(a, b):
+    return (a + b - 1) // b
+
+
+# ----------------------------------------------------------- raw entry points
+
+def fp8bw_quantize_rowwise(x, q, s, stream=None):
+    rows, cols = x.shape
+    _expect(x, torch.bfloat16, (rows, cols), "x")
+    _expect(q, torch.uint8, (rows, cols), "q")
+    _expect(s, torch.float32, (_cdiv(cols, 128), rows), "s")
+    _check(_lib.fp8bw_quantize_rowwise(_ptr(x), rows, cols, _ptr(q), _ptr(s),
+                                       _stream(stream)),
+           "fp8bw_quantize_rowwise")
+
+
+def fp8bw_quantize_colwise(x, q_t, s_t, q_row=None, s_row=None, stream=None):
+    rows, cols = x.shape
+    _expect(x, torch.bfloat16, (rows, cols), "x")
+    _expect(q_t, torch.uint8, (cols, rows), "q_t")
+    _expect(s_t, torch.float32, (_cdiv(rows, 128), cols), "s_t")
+    if q_row is not None:
+        _expect(q_row, torch.uint8, (rows, cols), "q_row")
+        _expect(s_row, torch.float32, (_cdiv(cols, 128), rows), "s_row")
+    _check(_lib.fp8bw_quantize_colwise(_ptr(x), rows, cols, _ptr(q_t),
+                                       _ptr(s_t), _ptr(q_row), _ptr(s_row),
+                                       _stream(stream)),
+           "fp8bw_quantize_colwise")
+
+
+def fp8bw_quantize_weight_block(w, q, s, q_t=None, stream=None):
+    n, k = w.shape
+    _expect(w, torch.bfloat16, (n, k), "w")
+    _expect(q, torch.uint8, (n, k), "q")
+    _expect(s, torch.float32, (_cdiv(n, 128), _cdiv(k, 128)), "s")
+    if q_t is not None:
+        _expect(q_t, torch.uint8, (k, n), "q_t")
+    _check(_lib.fp8bw_quantize_weight_block(_ptr(w), n, k, _ptr(q), _ptr(s),
+                                            _ptr(q_t), _stream(stream)),
+           "fp8bw_quantize_weight_block")
+
+
+def fp8bw_gemm_fprop(qx, sx, qw, sw, y, stream=None):
+    m, k = qx.shape
+    n = qw.shape[0]
+    _expect(qw, torch.uint8, (n, k), "qw")
+    _expect(sx, torch.float32, (_cdiv(k, 128), m), "sx")
+    _expect(sw, torch.float32, (_cdiv(n, 128), _cdiv(k, 128)), "sw")
+    _expect(y, torch.bfloat16, (m, n), "y")
+    _check(_lib.fp8bw_gemm_fprop(_ptr(qx), _ptr(sx), _ptr(qw), _ptr(sw), m, n,
+                                 k, _ptr(y), _stream(stream)),
+           "fp8bw_gemm_fprop")
+
+
+def fp8bw_gemm_dgrad(qdy, sdy, qw, qw_is_transposed, sw, dx, stream=None):
+    m, n = qdy.shape
+    k = qw.shape[0] if qw_is_transposed else qw.shape[1]
+    _expect(qw, torch.uint8, (k, n) if qw_is_transposed else (n, k), "qw")
+    _expect(sdy, torch.float32, (_cdiv(n, 128), m), "sdy")
+    _expect(sw, torch.float32, (_cdiv(n, 128), _cdiv(k, 128)), "sw")
+    _expect(dx, torch.bfloat16, (m, k), "dx")
+    _check(_lib.fp8bw_gemm_dgrad(_ptr(qdy), _ptr(sdy), _ptr(qw),
+                                 1 if qw_is_transposed else 0, _ptr(sw), m, n,
+                                 k, _ptr(dx), _stream(stream)),
+           "fp8bw_gemm_dgrad")
+
+
+def fp8bw_gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t, dw, stream=None):
+    n, m = qdy_t.shape
+    k = qx_t.shape[0]
+    _expect(qx_t, torch.uint8, (k, m), "qx_t")
+    _expect(sdy_t, torch.float32, (_cdiv(m, 128), n), "sdy_t")
+    _expect(sx_t, torch.float32, (_cdiv(m, 128), k), "sx_t")
+    _expect(dw, torch.bfloat16, (n, k), "dw")
+    _check(_lib.fp8bw_gemm_wgrad(_ptr(qdy_t), _ptr(sdy_t), _ptr(qx_t),
+                                 _ptr(sx_t), m, n, k, _ptr(dw),
+                                 _stream(stream)),
+           "fp8bw_gemm_wgrad")
+
+
+def fp8bw_check_device_error(stream=None):
+    _check(_lib.fp8bw_check_device_error(_stream(stream)),
+           "fp8bw_check_device_error")
+
+
+# ----------------------------------------------------------- allocating helpers
+
+def quantize_rowwise(x, stream=None):
+    rows, cols = x.shape
+    q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    s = torch.empty((_cdiv(cols, 128), rows), dtype=torch.float32,
+                    device=x.device)
+    fp8bw_quantize_rowwise(x, q, s, stream)
+    return q, s
+
+
+def quantize_colwise(x, with_rowwise=False, stream=None):
+    """-> (q_t, s_t) or (q_t, s_t, q_row, s_row) when with_rowwise."""
+    rows, cols = x.shape
+    dev = x.device
+    q_t = torch.empty((cols, rows), dtype=torch.uint8, device=dev)
+    s_t = torch.empty((_cdiv(rows, 128), cols), dtype=torch.float32,
+                      device=dev)
+    q_row = s_row = None
+    if with_rowwise:
+        q_row = torch.empty((rows, cols), dtype=torch.uint8, device=dev)
+        s_row = torch.empty((_cdiv(cols, 128), rows), dtype=torch.float32,
+                            device=dev)
+    fp8bw_quantize_colwise(x, q_t, s_t, q_row, s_row, stream)
+    return (q_t, s_t, q_row, s_row) if with_rowwise else (q_t, s_t)
+
+
+def quantize_weight_block(w, transposed=True, stream=None):
+    n, k = w.shape
+    dev = w.device
+    q = torch.empty((n, k), dtype=torch.uint8, device=dev)
+    s = torch.empty((_cdiv(n, 128), _cdiv(k, 128)), dtype=torch.float32,
+                    device=dev)
+    q_t = torch.empty((k, n), dtype=torch.uint8, device=dev) if transposed \
+        else None
+    fp8bw_quantize_weight_block(w, q, s, q_t, stream)
+    return q, s, q_t
+
+
+def gemm_fprop(qx, sx, qw, sw, stream=None):
+    y = torch.empty((qx.shape[0], qw.shape[0]), dtype=torch.bfloat16,
+                    device=qx.device)
+    fp8bw_gemm_fprop(qx, sx, qw, sw, y, stream)
+    return y
+
+
+def gemm_dgrad(qdy, sdy, qw, sw, qw_is_transposed=True, stream=None):
+    k = qw.shape[0] if qw_is_transposed else qw.shape[1]
+    dx = torch.empty((qdy.shape[0], k), dtype=torch.bfloat16,
+                     device=qdy.device)
+    fp8bw_gemm_dgrad(qdy, sdy, qw, qw_is_transposed, sw, dx, stream)
+    return dx
+
+
+def gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t, stream=None):
+    dw = torch.empty((qdy_t.shape[0], qx_t.shape[0]), dtype=torch.bfloat16,
+                     device=qdy_t.device)
+    fp8bw_gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t, dw, stream)
+    return dw

@@ -1,0 +1,157 @@
+/*
+ * fp8bw.h -- C ABI of the blockwise-FP8 training-linear library for B200
+ * (sm_100a).
+ *
+ * What the library computes (Puro-2B report summaries):
+ *   - arxiv-wiki summary of "Puro-2B: Poor Lab's Qwen2-1.5B Trained on RTX
+ *     5090 within $5090", section "Approach", item (4): the Transformer's main
+ *     linear operations run in blockwise FP8 E4M3, activations with one scale
+ *     per 1-D group of 128 elements, weights with one scale per 128x128 block.
+ *   - paperlayer.ai summary of the same report, Appendix C, "FP8
+ *     implementation pipeline": the E4M3 GEMMs of the linear layers are forward
+ *     propagation, data-gradient and weight-gradient; hidden/residual flow stays
+ *     bf16.
+ * The pages print no formula. The readings taken here:
+ *   - group scale: amax = max |x| over the group; qscale = 448/amax and stored
+ *     (dequantisation) scale s = amax/448, both fp32 round-to-nearest-even;
+ *     amax == 0, or a qscale that overflows fp32, gives qscale = s = 1.
+ *   - code = E4M3(x * qscale): one fp32 multiply, then round-to-nearest-even
+ *     with saturation to +-448 (0x7E/0xFE).
+ *   - GEMMs accumulate in fp32; every 128-long chunk of the contraction
+ *     dimension is computed separately on the tensor cores and added into the
+ *     fp32 accumulator times the product of its two scales; bf16 output (RNE).
+ *
+ * Conventions for every call:
+ *   - All data pointers are DEVICE pointers owned by the caller. The library
+ *     never allocates, frees or keeps them. Outputs must not alias inputs. A
+ *     pointer may be NULL only when its buffer holds no element.
+ *   - bf16 tensors are passed as uint16_t bit patterns. FP8 codes are uint8_t
+ *     OCP E4M3 codes. Scales are fp32.
+ *   - Matrices are dense row-major (leading dimension = row length).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t, NULL = legacy
+ *     default stream) and returns an fp8bw_status. Argument errors are found
+ *     on the host before anything is launched, and then nothing is written.
+ *   - Shapes: every dimension >= 0 and a multiple of 16. Dimensions that are
+ *     not multiples of 128 give a short last group (its amax runs over the
+ *     elements present) and a short last chunk. A zero dimension is a no-op,
+ *     except a GEMM with an empty contraction, which writes zeros.
+ *   - Pointers must be 16-byte aligned.
+ *   - Scale layouts ("group-major, contiguous along the other dimension", so a
+ *     128-row GEMM tile reads its 128 scales of one chunk in one 512-B run):
+ *       row-wise 1x128 groups of X[rows, cols]  : s[ceil(cols/128)][rows]
+ *       col-wise 128x1 groups of X[rows, cols]  : s_t[ceil(rows/128)][cols]
+ *       128x128 blocks of W[n, k]               : s[ceil(n/128)][ceil(k/128)]
+ *   - The kernels run only on compute capability 10.0 (B200, sm_100a); other
+ *     devices get FP8BW_ERR_DEVICE.
+ *   - Device-side waits are bounded: a wait that does not finish within about
+ *     two seconds makes the kernel record FP8BW_ERR_DEVICE_TIMEOUT in a device
+ *     flag and return; fp8bw_check_device_error() reads and clears that flag.
+ */
+#ifndef FP8BW_H
+#define FP8BW_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fp8bw_status {
+    FP8BW_OK = 0,
+    FP8BW_ERR_NULL = -1,           /* a required pointer is NULL */
+    FP8BW_ERR_SHAPE = -2,          /* a dimension < 0 or not a multiple of 16 */
+    FP8BW_ERR_ALIGN = -3,          /* a pointer is not 16-byte aligned */
+    FP8BW_ERR_DEVICE = -4,         /* current device is not sm_100 */
+    FP8BW_ERR_LAUNCH = -5,         /* the CUDA launch failed */
+    FP8BW_ERR_DEVICE_TIMEOUT = -6, /* a bounded device-side wait expired */
+    FP8BW_ERR_CUDA = -7,           /* another CUDA runtime/driver call failed */
+    FP8BW_ERR_ALIAS = -8           /* an output overlaps an input */
+} fp8bw_status;
+
+/* Row-wise 1x128 quantisation of an activation or gradient X[rows, cols]
+ * (groups along cols, the contraction dimension of fprop for X and of dgrad
+ * for dY).
+ *   x : bf16 [rows, cols]                         (in)
+ *   q : E4M3 codes [rows, cols]                   (out)
+ *   s : fp32 scales [ceil(cols/128)][rows]        (out)
+ * Source: arxiv-wiki summary, Approach item (4) (activation 1-D groups of 128).
+ * HBM traffic: 2 B read + 1 B + 4/128 B written per element. */
+int fp8bw_quantize_rowwise(const uint16_t* x, int64_t rows, int64_t cols,
+                           uint8_t* q, float* s, void* stream);
+
+/* Column-wise 128x1 quantisation of X[rows, cols] (groups along rows, the
+ * token dimension, which the weight-gradient GEMM contracts), with the codes
+ * written transposed. If q_row and s_row are both non-NULL the same pass also
+ * writes the row-wise 1x128 result (one read of X for both).
+ *   x     : bf16 [rows, cols]                     (in)
+ *   q_t   : E4M3 codes [cols, rows]               (out)
+ *   s_t   : fp32 scales [ceil(rows/128)][cols]    (out)
+ *   q_row : E4M3 codes [rows, cols] or NULL       (out)
+ *   s_row : fp32 [ceil(cols/128)][rows] or NULL   (out)
+ * Source: paperlayer.ai summary, Appendix C, "FP8 implementation pipeline"
+ * (weight-gradient GEMM) with the 1-D group of 128 of the arxiv-wiki summary,
+ * Approach item (4). Either both of q_row/s_row are NULL or neither. */
+int fp8bw_quantize_colwise(const uint16_t* x, int64_t rows, int64_t cols,
+                           uint8_t* q_t, float* s_t, uint8_t* q_row,
+                           float* s_row, void* stream);
+
+/* 128x128 block quantisation of a weight W[n, k] (out x in).
+ *   w   : bf16 [n, k]                             (in)
+ *   q   : E4M3 codes [n, k]                       (out)
+ *   s   : fp32 scales [ceil(n/128)][ceil(k/128)]  (out)
+ *   q_t : E4M3 codes [k, n] (the same codes transposed, for dgrad) or NULL
+ * Source: arxiv-wiki summary, Approach item (4) (weights in 128x128 blocks). */
+int fp8bw_quantize_weight_block(const uint16_t* w, int64_t n, int64_t k,
+                                uint8_t* q, float* s, uint8_t* q_t,
+                                void* stream);
+
+/* fprop: Y[m, n] = bf16( sum_c sX[c][m] * sW[n/128][c] *
+ *                        sum_{kk in chunk c} qX[m, kk] * qW[n, kk] )
+ *   qx, sx : row-wise quantised X: [m, k], [ceil(k/128)][m]
+ *   qw, sw : block-quantised W: [n, k], [ceil(n/128)][ceil(k/128)]
+ *   y      : bf16 [m, n]                          (out)
+ * Source: paperlayer.ai summary, Appendix C ("forward propagation"). */
+int fp8bw_gemm_fprop(const uint8_t* qx, const float* sx, const uint8_t* qw,
+                     const float* sw, int64_t m, int64_t n, int64_t k,
+                     uint16_t* y, void* stream);
+
+/* dgrad: dX[m, k] = bf16( sum_c sdY[c][m] * sW[c][k/128] *
+ *                         sum_{nn in chunk c} qdY[m, nn] * qW[nn, k] )
+ *   qdy, sdy : row-wise quantised dY: [m, n], [ceil(n/128)][m]
+ *   qw       : the weight codes, either transposed qW^T [k, n]
+ *              (qw_is_transposed = 1, as written by fp8bw_quantize_weight_block
+ *              into q_t) or as stored, qW [n, k] (qw_is_transposed = 0)
+ *   sw       : block scales [ceil(n/128)][ceil(k/128)] (the same blocks as
+ *              fprop: a square block is transpose invariant)
+ *   dx       : bf16 [m, k]                        (out)
+ * Source: paperlayer.ai summary, Appendix C ("data-gradient"). */
+int fp8bw_gemm_dgrad(const uint8_t* qdy, const float* sdy, const uint8_t* qw,
+                     int qw_is_transposed, const float* sw, int64_t m,
+                     int64_t n, int64_t k, uint16_t* dx, void* stream);
+
+/* wgrad: dW[n, k] = bf16( sum_c sdYt[c][n] * sXt[c][k] *
+ *                         sum_{mm in chunk c} qdYt[n, mm] * qXt[k, mm] )
+ *   qdy_t, sdy_t : col-wise quantised dY: [n, m], [ceil(m/128)][n]
+ *   qx_t,  sx_t  : col-wise quantised X:  [k, m], [ceil(m/128)][k]
+ *   dw           : bf16 [n, k]                    (out)
+ * Source: paperlayer.ai summary, Appendix C ("weight-gradient"). */
+int fp8bw_gemm_wgrad(const uint8_t* qdy_t, const float* sdy_t,
+                     const uint8_t* qx_t, const float* sx_t, int64_t m,
+                     int64_t n, int64_t k, uint16_t* dw, void* stream);
+
+/* Synchronises `stream`, then returns FP8BW_ERR_DEVICE_TIMEOUT if any kernel
+ * of this library on the current device recorded an expired wait since the
+ * last call (and clears the record), else FP8BW_OK (or FP8BW_ERR_CUDA if the
+ * synchronisation itself failed). */
+int fp8bw_check_device_error(void* stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char* fp8bw_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int fp8bw_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FP8BW_H */

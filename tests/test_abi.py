@@ -1,0 +1,117 @@
+"""The C ABI without a GPU: every symbol declared in include/fp8bw.h is
+exported by libfp8bw.so, and the host-side argument checks reject bad calls
+before anything touches the device (fake pointer values are never
+dereferenced because each call below fails validation first)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from blockwise_fp8_linear_fp8bw_b200 import _native
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp8bw.h")
+
+OK, E_NULL, E_SHAPE, E_ALIGN, E_DEVICE, E_LAUNCH, E_TIMEOUT, E_CUDA, E_ALIAS = \
+    0, -1, -2, -3, -4, -5, -6, -7, -8
+
+A = 0x10000000   # fake, 16-byte aligned, never dereferenced
+B = 0x20000000
+C = 0x30000000
+D = 0x40000000
+E = 0x50000000
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fp8bw_[a-z_0-9]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return _native.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) == 9
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(_native.SIGNATURES)
+
+
+def test_status_strings_and_version(lib):
+    assert lib.fp8bw_version() == 100
+    for st in (OK, E_NULL, E_SHAPE, E_ALIGN, E_DEVICE, E_LAUNCH, E_TIMEOUT,
+               E_CUDA, E_ALIAS):
+        s = lib.fp8bw_status_string(st).decode()
+        assert s and s != "unknown status"
+    assert lib.fp8bw_status_string(12345).decode() == "unknown status"
+
+
+def test_null_pointers_rejected(lib):
+    assert lib.fp8bw_quantize_rowwise(None, 128, 128, B, C, None) == E_NULL
+    assert lib.fp8bw_quantize_colwise(A, 128, 128, None, C, None, None,
+                                      None) == E_NULL
+    # q_row without s_row
+    assert lib.fp8bw_quantize_colwise(A, 128, 128, B, C, D, None,
+                                      None) == E_NULL
+    assert lib.fp8bw_quantize_weight_block(A, 128, 128, None, C, None,
+                                           None) == E_NULL
+    assert lib.fp8bw_gemm_fprop(A, B, C, None, 128, 128, 128, E,
+                                None) == E_NULL
+    assert lib.fp8bw_gemm_dgrad(A, B, None, 1, D, 128, 128, 128, E,
+                                None) == E_NULL
+    assert lib.fp8bw_gemm_wgrad(A, B, C, D, 128, 128, 128, None,
+                                None) == E_NULL
+
+
+@pytest.mark.parametrize("rows,cols", [(-16, 128), (128, -16), (100, 128),
+                                       (128, 8), (128, 130), (1 << 31, 16)])
+def test_bad_shapes_rejected(lib, rows, cols):
+    assert lib.fp8bw_quantize_rowwise(A, rows, cols, B, C, None) == E_SHAPE
+    assert lib.fp8bw_quantize_colwise(A, rows, cols, B, C, None, None,
+                                      None) == E_SHAPE
+    assert lib.fp8bw_quantize_weight_block(A, rows, cols, B, C, None,
+                                           None) == E_SHAPE
+    assert lib.fp8bw_gemm_fprop(A, B, C, D, rows, cols, 128, E,
+                                None) == E_SHAPE
+    assert lib.fp8bw_gemm_dgrad(A, B, C, 0, D, 128, rows, cols, E,
+                                None) == E_SHAPE
+    assert lib.fp8bw_gemm_wgrad(A, B, C, D, cols, 128, rows, E,
+                                None) == E_SHAPE
+
+
+def test_misaligned_pointers_rejected(lib):
+    assert lib.fp8bw_quantize_rowwise(A + 2, 128, 128, B, C, None) == E_ALIGN
+    assert lib.fp8bw_quantize_colwise(A, 128, 128, B, C + 4, None, None,
+                                      None) == E_ALIGN
+    assert lib.fp8bw_quantize_weight_block(A, 128, 128, B, C, D + 8,
+                                           None) == E_ALIGN
+    assert lib.fp8bw_gemm_fprop(A, B + 1, C, D, 128, 128, 128, E,
+                                None) == E_ALIGN
+    assert lib.fp8bw_gemm_dgrad(A, B, C, 1, D, 128, 128, 128, E + 2,
+                                None) == E_ALIGN
+    assert lib.fp8bw_gemm_wgrad(A, B, C, D + 4, 128, 128, 128, E,
+                                None) == E_ALIGN
+
+
+def test_aliased_outputs_rejected(lib):
+    # output codes overlapping the bf16 input
+    assert lib.fp8bw_quantize_rowwise(A, 128, 128, A + 16, C, None) == E_ALIAS
+    # GEMM output on top of the scales
+    assert lib.fp8bw_gemm_fprop(A, B, C, D, 128, 128, 128, B,
+                                None) == E_ALIAS
+    assert lib.fp8bw_gemm_wgrad(A, B, C, D, 128, 128, 128, C + 256,
+                                None) == E_ALIAS
+
+
+@pytest.mark.skipif(
+    __import__("torch").cuda.is_available(),
+    reason="checks the no-device path; on a GPU host the call would launch")
+def test_valid_call_without_device_reports_device_error(lib):
+    assert lib.fp8bw_quantize_rowwise(A, 128, 128, B, C, None) == E_DEVICE
+    assert lib.fp8bw_gemm_fprop(A, B, C, D, 128, 128, 128, E,
+                                None) == E_DEVICE
