@@ -44,6 +44,7 @@ import numpy as np  # noqa: E402
 
 WORKLOAD = "stack28_m16384"
 LAYERS = 28
+KINDS = ("qkv", "o", "gate_up", "down")
 TOKENS = 16384
 METRIC = ("blockwise-FP8 GEMM TFLOP/s (fwd/dgrad/wgrad) & % FP8 peak; "
           "quantize GB/s % HBM")
@@ -60,13 +61,20 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    return p.parse_args()
+    p.add_argument("--layers", type=int, default=28,
+                   help="layers per step (profiling runs use fewer)")
+    p.add_argument("--linears", default="qkv,o,gate_up,down",
+                   help="comma list of the linears in a layer")
+    args = p.parse_args()
+    global LAYERS, KINDS
+    LAYERS = args.layers
+    KINDS = tuple(args.linears.split(","))
+    return args
 
 
 def kinds():
     from synthetic import LINEARS
-    return [(kind, LINEARS[kind][0], LINEARS[kind][1])
-            for kind in ("qkv", "o", "gate_up", "down")]
+    return [(kind, LINEARS[kind][0], LINEARS[kind][1]) for kind in KINDS]
 
 
 def step_gemm_flops():
@@ -496,7 +504,9 @@ def run_gpu(args):
         "vs_baseline": None,
         "dtype": "e4m3",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "layers": LAYERS, "tokens": TOKENS,
+        "config": {"workload": WORKLOAD if (LAYERS, KINDS) == (28, (
+                       "qkv", "o", "gate_up", "down")) else "partial",
+                   "layers": LAYERS, "tokens": TOKENS,
                    "linears": {kd: [k, n] for kd, k, n in kinds()},
                    "gemm_tflop_per_step": flops / 1e12,
                    "l2": "inputs larger than L2 (>1 GB streamed between "

@@ -102,6 +102,22 @@ int encode_u8_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t ou
   return r == CUDA_SUCCESS ? FP8BW_OK : FP8BW_ERR_CUDA;
 }
 
+// 2-D bf16 output tensor [rows, cols] written in 32 x 32 boxes (64-byte rows,
+// 64-byte swizzle); out-of-range parts of a box are not written.
+int encode_bf16_out(CUtensorMap* map, void* base, uint64_t cols, uint64_t rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  int st = get_encode(&enc);
+  if (st != FP8BW_OK) return st;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {32u, 32u};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FP8BW_OK : FP8BW_ERR_CUDA;
+}
+
 // --------------------------------------------------------------- GEMM launch
 struct GemmProblem {
   const uint8_t* a;  // [mo][kc]
@@ -139,7 +155,7 @@ int launch_gemm_t(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t stre
   });
   if (prep_status != FP8BW_OK) return prep_status;
 
-  CUtensorMap tm_a, tm_b;
+  CUtensorMap tm_a, tm_b, tm_out;
   int st = encode_u8_2d(&tm_a, p.a, static_cast<uint64_t>(p.kc), static_cast<uint64_t>(p.mo),
                         gemm::BM);
   if (st != FP8BW_OK) return st;
@@ -147,6 +163,8 @@ int launch_gemm_t(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t stre
     st = encode_u8_2d(&tm_b, p.b, static_cast<uint64_t>(p.no), static_cast<uint64_t>(p.kc), 128);
   else
     st = encode_u8_2d(&tm_b, p.b, static_cast<uint64_t>(p.kc), static_cast<uint64_t>(p.no), BN);
+  if (st != FP8BW_OK) return st;
+  st = encode_bf16_out(&tm_out, p.out, static_cast<uint64_t>(p.no), static_cast<uint64_t>(p.mo));
   if (st != FP8BW_OK) return st;
 
   gemm::Args g;
@@ -164,7 +182,7 @@ int launch_gemm_t(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t stre
   g.out = p.out;
   const int tiles = g.tiles_m * g.tiles_n;
   const int grid = std::min(tiles, dev.sm_count);
-  kernel<<<grid, gemm::kThreads, L::kAlloc, stream>>>(tm_a, tm_b, g);
+  kernel<<<grid, gemm::kThreads, L::kAlloc, stream>>>(tm_a, tm_b, tm_out, g);
   return cudaGetLastError() == cudaSuccess ? FP8BW_OK : FP8BW_ERR_LAUNCH;
 }
 

@@ -119,6 +119,63 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src,
       : "memory");
 }
 
+// Shared -> global tensor store (bulk async-group); OOB parts are clipped.
+__device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src,
+                                             int32_t x, int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], "
+      "[%3];" ::"l"(reinterpret_cast<uint64_t>(tmap)),
+      "r"(x), "r"(y), "r"(src)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Wait until all but `N` committed bulk groups have finished READING shared
+// memory (their buffers may then be overwritten).
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+// Wait until all committed bulk groups have completed.
+__device__ __forceinline__ void bulk_wait_group_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// Make this thread's generic-proxy shared-memory writes visible to the async
+// proxy (TMA) before a bulk copy reads them.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Packed fp32 pair arithmetic (one instruction, two IEEE round-to-nearest
+// results): a = x * s + a and p = x * y, element-wise on (lo, hi).
+__device__ __forceinline__ void ffma2(float& a0, float& a1, float x0, float x1,
+                                      float s0, float s1) {
+  asm("{\n\t.reg .b64 a, x, s;\n\t"
+      "mov.b64 a, {%0, %1};\n\t"
+      "mov.b64 x, {%2, %3};\n\t"
+      "mov.b64 s, {%4, %5};\n\t"
+      "fma.rn.f32x2 a, x, s, a;\n\t"
+      "mov.b64 {%0, %1}, a;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(x0), "f"(x1), "f"(s0), "f"(s1));
+}
+
+__device__ __forceinline__ void fmul2(float& p0, float& p1, float x0, float x1,
+                                      float y0, float y1) {
+  asm("{\n\t.reg .b64 p, x, y;\n\t"
+      "mov.b64 x, {%2, %3};\n\t"
+      "mov.b64 y, {%4, %5};\n\t"
+      "mul.rn.f32x2 p, x, y;\n\t"
+      "mov.b64 {%0, %1}, p;\n\t}"
+      : "=f"(p0), "=f"(p1)
+      : "f"(x0), "f"(x1), "f"(y0), "f"(y1));
+}
+
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(
                    reinterpret_cast<uint64_t>(tmap))

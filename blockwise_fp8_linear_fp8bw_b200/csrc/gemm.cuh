@@ -23,11 +23,13 @@
 //               writes the chunk's two block scales itself.
 //   warps 4-11  promotion / epilogue: warp w reads TMEM lanes 32*(w%4)..+31
 //               (its 32 output rows) and one half of the BN columns; per chunk
-//               it loads the partial sums with tcgen05.ld and adds them, times
-//               the two scales, into an fp32 accumulator held in registers
-//               (BN/2 per thread); after the last chunk it writes bf16 rows.
-// Registers: warps 0-3 drop to 56 per thread, the eight epilogue warps rise to
-// 224 (setmaxnreg); 4*32*56 + 8*32*224 = 384 * 168, the launch budget.
+//               it loads the partial sums with tcgen05.ld, hands the TMEM
+//               buffer back, and adds them, times the two scales, into an fp32
+//               accumulator held in registers (BN/2 per thread, packed f32x2
+//               FMAs); after the last chunk it converts to bf16, stages 32x32
+//               boxes in shared memory and writes them with TMA stores.
+// Registers: warps 0-3 drop to 40 per thread, the eight epilogue warps rise to
+// 232 (setmaxnreg); 4*32*40 + 8*32*232 = 384 * 168, the launch budget.
 // Every mbarrier wait is bounded (about 2 s, see common.cuh); on expiry the
 // CTA records the error, drains its outstanding copies and MMAs, frees TMEM
 // and exits.
@@ -48,9 +50,9 @@ constexpr int kScaleStages = 8;   // scale ring depth
 constexpr int kThreads = 384;
 constexpr int kFirstEpiWarp = 4;
 constexpr int kNumEpiWarps = 8;
-constexpr int kProducerRegs = 56;
-constexpr int kEpilogueRegs = 224;
-constexpr int kLaunchRegs = 168;  // (4*32*56 + 8*32*224) / 384
+constexpr int kProducerRegs = 40;
+constexpr int kEpilogueRegs = 232;
+constexpr int kLaunchRegs = 168;  // (4*32*40 + 8*32*232) / 384
 
 static_assert(4 * 32 * kProducerRegs + kNumEpiWarps * 32 * kEpilogueRegs ==
                   kThreads * kLaunchRegs,
@@ -70,7 +72,11 @@ struct Layout {
   // full[S], empty[S], sfull[SS], sempty[SS], tfull[2], tempty[2], drain
   static constexpr int kNumBars = 2 * kStages + 2 * kScaleStages + 5;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kBytes = kMiscOff + 16;
+  // per epilogue warp: a 32 x 32 bf16 box (2 KB, 64-byte swizzle) staged for
+  // the TMA store of the output
+  static constexpr int kOutWarpBytes = 32 * 32 * 2;
+  static constexpr int kOutOff = ((kMiscOff + 16 + 1023) / 1024) * 1024;
+  static constexpr int kBytes = kOutOff + kNumEpiWarps * kOutWarpBytes;
   static constexpr int kAlloc = kBytes + 1024;  // base is aligned up to 1024
   static constexpr uint32_t kTmemCols = 2 * BN;  // power of two for BN = 128/256
   static_assert(kBarOff % 8 == 0, "barrier alignment");
@@ -103,6 +109,7 @@ template <int BN, bool VEC_B, bool B_MN>
 __global__ void __launch_bounds__(kThreads, 1)
     blockwise_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
                           const __grid_constant__ CUtensorMap tm_b,
+                          const __grid_constant__ CUtensorMap tm_out,
                           const Args g) {
   using L = Layout<BN, VEC_B>;
   constexpr int kHalf = BN / 2;                      // columns per epilogue thread
@@ -146,6 +153,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tm_a);
     prefetch_tmap(&tm_b);
+    prefetch_tmap(&tm_out);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), L::kTmemCols);
@@ -312,10 +320,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ promotion + epilogue
     setmaxnreg_inc();
     const int q = warp & 3;                          // TMEM lane quarter
-    const int h = (warp - kFirstEpiWarp) >> 2;       // column half of the tile
+    const int ew = warp - kFirstEpiWarp;
+    const int h = ew >> 2;                           // column half of the tile
     const int row = q * 32 + lane;                   // tile row = TMEM lane
+    const uint32_t stage_out = sbase + L::kOutOff + ew * L::kOutWarpBytes;
     uint32_t tc = 0, sit = 0;
-    bool ok = true;
+    bool ok = true, store_pending = false;
     for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
       const int tm = tile / g.tiles_n, tn = tile % g.tiles_n;
       float acc[kHalf];
@@ -342,63 +352,75 @@ __global__ void __launch_bounds__(kThreads, 1)
                                static_cast<uint32_t>(tb * BN + h * kHalf);
 #pragma unroll
         for (int part = 0; part < kHalf / 64; ++part) {
-          uint32_t r0[32], r1[32];
-          tmem_ld32(taddr + part * 64, r0);
-          tmem_ld32(taddr + part * 64 + 32, r1);
+          uint32_t r[64];
+          tmem_ld32(taddr + part * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+          tmem_ld32(taddr + part * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
           tmem_wait_ld();
+          if (part == kHalf / 64 - 1) {
+            // Every TMEM read of this chunk has landed: hand the buffer back to
+            // the MMA warp before doing the arithmetic.
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty_bar(tb));
+          }
+          float* a = acc + part * 64;
           if constexpr (VEC_B) {
             const float* sbp = sbv + h * kHalf + part * 64;
 #pragma unroll
-            for (int j = 0; j < 32; j += 4) {
+            for (int j = 0; j < 64; j += 4) {
               const float4 b4 = *reinterpret_cast<const float4*>(sbp + j);
-              acc[part * 64 + j + 0] = fmaf(__uint_as_float(r0[j + 0]), sa_v * b4.x, acc[part * 64 + j + 0]);
-              acc[part * 64 + j + 1] = fmaf(__uint_as_float(r0[j + 1]), sa_v * b4.y, acc[part * 64 + j + 1]);
-              acc[part * 64 + j + 2] = fmaf(__uint_as_float(r0[j + 2]), sa_v * b4.z, acc[part * 64 + j + 2]);
-              acc[part * 64 + j + 3] = fmaf(__uint_as_float(r0[j + 3]), sa_v * b4.w, acc[part * 64 + j + 3]);
-            }
-#pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-              const float4 b4 = *reinterpret_cast<const float4*>(sbp + 32 + j);
-              acc[part * 64 + 32 + j + 0] = fmaf(__uint_as_float(r1[j + 0]), sa_v * b4.x, acc[part * 64 + 32 + j + 0]);
-              acc[part * 64 + 32 + j + 1] = fmaf(__uint_as_float(r1[j + 1]), sa_v * b4.y, acc[part * 64 + 32 + j + 1]);
-              acc[part * 64 + 32 + j + 2] = fmaf(__uint_as_float(r1[j + 2]), sa_v * b4.z, acc[part * 64 + 32 + j + 2]);
-              acc[part * 64 + 32 + j + 3] = fmaf(__uint_as_float(r1[j + 3]), sa_v * b4.w, acc[part * 64 + 32 + j + 3]);
+              float w0, w1, w2, w3;
+              fmul2(w0, w1, sa_v, sa_v, b4.x, b4.y);
+              fmul2(w2, w3, sa_v, sa_v, b4.z, b4.w);
+              ffma2(a[j], a[j + 1], __uint_as_float(r[j]), __uint_as_float(r[j + 1]), w0, w1);
+              ffma2(a[j + 2], a[j + 3], __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]), w2, w3);
             }
           } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              acc[part * 64 + j] = fmaf(__uint_as_float(r0[j]), blk_scale, acc[part * 64 + j]);
-              acc[part * 64 + 32 + j] = fmaf(__uint_as_float(r1[j]), blk_scale, acc[part * 64 + 32 + j]);
-            }
+            for (int j = 0; j < 64; j += 2)
+              ffma2(a[j], a[j + 1], __uint_as_float(r[j]), __uint_as_float(r[j + 1]),
+                    blk_scale, blk_scale);
           }
         }
-        tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(tempty_bar(tb));
-          mbar_arrive(sempty_bar(ss));
-        }
+        if (lane == 0) mbar_arrive(sempty_bar(ss));
       }
       if (!ok) break;
 
-      // ---- bf16 output: this thread's row, columns [n0 + h*kHalf, +kHalf)
-      const int grow = tm * BM + row;
-      const int gcol0 = tn * BN + h * kHalf;
-      if (grow < g.mo) {
-        uint16_t* dst = g.out + static_cast<int64_t>(grow) * g.no + gcol0;
+      // ---- bf16 output through shared memory and TMA stores: this warp owns
+      // rows [m0 + 32q, +32) and columns [n0 + h*kHalf, +kHalf), written as
+      // 32 x 32 boxes (64-byte rows, 16-byte chunks xor-swizzled by row/2).
+      const int y0 = tm * BM + q * 32;
+      const int x0 = tn * BN + h * kHalf;
 #pragma unroll
-        for (int j = 0; j < kHalf; j += 8) {
-          if (gcol0 + j < g.no) {
-            uint4 v;
-            v.x = pack_bf16x2(acc[j + 0], acc[j + 1]);
-            v.y = pack_bf16x2(acc[j + 2], acc[j + 3]);
-            v.z = pack_bf16x2(acc[j + 4], acc[j + 5]);
-            v.w = pack_bf16x2(acc[j + 6], acc[j + 7]);
-            *reinterpret_cast<uint4*>(dst + j) = v;
-          }
+      for (int gi = 0; gi < kHalf / 32; ++gi) {
+        if (x0 + gi * 32 >= g.no || y0 >= g.mo) continue;
+        if (store_pending) {
+          if (lane == 0) bulk_wait_group_read<0>();
+          __syncwarp();
         }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float* v = acc + gi * 32 + j * 8;
+          const uint32_t w0 = pack_bf16x2(v[0], v[1]);
+          const uint32_t w1 = pack_bf16x2(v[2], v[3]);
+          const uint32_t w2 = pack_bf16x2(v[4], v[5]);
+          const uint32_t w3 = pack_bf16x2(v[6], v[7]);
+          const uint32_t dst = stage_out + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(w0),
+                       "r"(w1), "r"(w2), "r"(w3)
+                       : "memory");
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tm_out, stage_out, x0 + gi * 32, y0);
+          bulk_commit_group();
+        }
+        store_pending = true;
       }
     }
+    if (lane == 0) bulk_wait_group_all();
   }
 
   tc_fence_before();
