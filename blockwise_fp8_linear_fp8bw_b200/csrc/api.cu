@@ -12,8 +12,15 @@
 #include <mutex>
 
 #include "common.cuh"
-#include "gemm.cuh"
+#include "gemm_pair.cuh"
 #include "quant.cuh"
+
+#ifndef GEMM_BN_BLOCK
+#define GEMM_BN_BLOCK 256
+#endif
+#ifndef GEMM_BN_VEC
+#define GEMM_BN_VEC 256
+#endif
 
 namespace fp8bw {
 
@@ -102,6 +109,24 @@ int encode_u8_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t ou
   return r == CUDA_SUCCESS ? FP8BW_OK : FP8BW_ERR_CUDA;
 }
 
+}  // namespace
+
+int encode_bf16_in(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  int st = get_encode(&enc);
+  if (st != FP8BW_OK) return st;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {128u, 128u};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FP8BW_OK : FP8BW_ERR_CUDA;
+}
+
+namespace {
+
 // 2-D bf16 output tensor [rows, cols] written in 32 x 32 boxes (64-byte rows,
 // 64-byte swizzle); out-of-range parts of a box are not written.
 int encode_bf16_out(CUtensorMap* map, void* base, uint64_t cols, uint64_t rows) {
@@ -131,26 +156,42 @@ struct GemmProblem {
   uint16_t* out;
 };
 
+// CTA-pair kernel: 256 x 256 output tiles on clusters of two CTAs.
 template <int BN, bool VEC_B, bool B_MN>
-int launch_gemm_t(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t stream) {
-  using L = gemm::Layout<BN, VEC_B>;
-  auto kernel = gemm::blockwise_gemm_kernel<BN, VEC_B, B_MN>;
+int launch_gemm_pair(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t stream) {
+  using L = gemm::PairLayout<BN, VEC_B>;
+  auto kernel = gemm::blockwise_gemm_pair_kernel<BN, VEC_B, B_MN>;
   static std::once_flag once;
   static int prep_status = FP8BW_OK;
+  static int max_clusters = 0;
   std::call_once(once, [&]() {
     cudaFuncAttributes attr;
-    if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess) {
+    // With BN = 256 the kernel redistributes registers with setmaxnreg, which
+    // draws on exactly the launch allocation: refuse to launch if that
+    // allocation is smaller than the split assumes.
+    if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess ||
+        (BN == 256 && attr.numRegs < gemm::kLaunchRegs)) {
       prep_status = FP8BW_ERR_LAUNCH;
       return;
     }
-    // setmaxnreg redistributes exactly the registers the CTA was launched
-    // with; a smaller launch allocation would make the increase wait forever.
-    if (attr.numRegs < gemm::kLaunchRegs) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) !=
+        cudaSuccess) {
       prep_status = FP8BW_ERR_LAUNCH;
       return;
     }
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             L::kAlloc) != cudaSuccess)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * dev.sm_count, 1, 1);
+    cfg.blockDim = dim3(gemm::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = L::kAlloc;
+    cudaLaunchAttribute attr_cl;
+    attr_cl.id = cudaLaunchAttributeClusterDimension;
+    attr_cl.val.clusterDim.x = 2;
+    attr_cl.val.clusterDim.y = 1;
+    attr_cl.val.clusterDim.z = 1;
+    cfg.attrs = &attr_cl;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&max_clusters, kernel, &cfg) != cudaSuccess ||
+        max_clusters < 1)
       prep_status = FP8BW_ERR_LAUNCH;
   });
   if (prep_status != FP8BW_OK) return prep_status;
@@ -162,7 +203,8 @@ int launch_gemm_t(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t stre
   if (B_MN)
     st = encode_u8_2d(&tm_b, p.b, static_cast<uint64_t>(p.no), static_cast<uint64_t>(p.kc), 128);
   else
-    st = encode_u8_2d(&tm_b, p.b, static_cast<uint64_t>(p.kc), static_cast<uint64_t>(p.no), BN);
+    st = encode_u8_2d(&tm_b, p.b, static_cast<uint64_t>(p.kc), static_cast<uint64_t>(p.no),
+                      BN / 2);
   if (st != FP8BW_OK) return st;
   st = encode_bf16_out(&tm_out, p.out, static_cast<uint64_t>(p.no), static_cast<uint64_t>(p.mo));
   if (st != FP8BW_OK) return st;
@@ -171,8 +213,8 @@ int launch_gemm_t(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t stre
   g.mo = static_cast<int>(p.mo);
   g.no = static_cast<int>(p.no);
   g.kc = static_cast<int>(p.kc);
-  g.tiles_m = static_cast<int>(cdiv(p.mo, gemm::BM));
-  g.tiles_n = static_cast<int>(cdiv(p.no, BN));
+  g.tiles_m = static_cast<int>(cdiv(p.mo, 2 * gemm::BM));
+  g.tiles_n = static_cast<int>(cdiv(p.no, L::BN));
   g.chunks = static_cast<int>(cdiv(p.kc, gemm::BK));
   g.sa = p.sa;
   g.sb = p.sb;
@@ -180,9 +222,9 @@ int launch_gemm_t(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t stre
   g.sbc = p.sbc;
   g.nblk = static_cast<int>(cdiv(p.no, 128));
   g.out = p.out;
-  const int tiles = g.tiles_m * g.tiles_n;
-  const int grid = std::min(tiles, dev.sm_count);
-  kernel<<<grid, gemm::kThreads, L::kAlloc, stream>>>(tm_a, tm_b, tm_out, g);
+  const int64_t tiles = static_cast<int64_t>(g.tiles_m) * g.tiles_n;
+  const int clusters = static_cast<int>(std::min<int64_t>(tiles, max_clusters));
+  kernel<<<2 * clusters, gemm::kThreads, L::kAlloc, stream>>>(tm_a, tm_b, tm_out, g);
   return cudaGetLastError() == cudaSuccess ? FP8BW_OK : FP8BW_ERR_LAUNCH;
 }
 
@@ -196,9 +238,10 @@ int run_gemm(const GemmProblem& p, cudaStream_t stream) {
                ? FP8BW_OK
                : FP8BW_ERR_CUDA;
   }
-  if (p.vec_b) return launch_gemm_t<256, true, false>(p, dev, stream);
-  if (p.b_mn) return launch_gemm_t<256, false, true>(p, dev, stream);
-  return launch_gemm_t<256, false, false>(p, dev, stream);
+  if (cdiv(p.mo, 256) * cdiv(p.no, 256) > (int64_t(1) << 30)) return FP8BW_ERR_SHAPE;
+  if (p.vec_b) return launch_gemm_pair<GEMM_BN_VEC, true, false>(p, dev, stream);
+  if (p.b_mn) return launch_gemm_pair<256, false, true>(p, dev, stream);
+  return launch_gemm_pair<GEMM_BN_BLOCK, false, false>(p, dev, stream);
 }
 
 }  // namespace
@@ -238,10 +281,8 @@ int fp8bw_quantize_rowwise(const uint16_t* x, int64_t rows, int64_t cols, uint8_
   int st = current_device_info(&dev);
   if (st != FP8BW_OK) return st;
   if (rows == 0 || cols == 0) return FP8BW_OK;
-  return launch_quantize(kModeRow, x, rows, cols, q, s, nullptr, nullptr, nullptr,
-                         static_cast<cudaStream_t>(stream)) == cudaSuccess
-             ? FP8BW_OK
-             : FP8BW_ERR_LAUNCH;
+  return launch_quantize(kModeRow, x, rows, cols, q, s, nullptr, nullptr, nullptr, dev.sm_count,
+                         static_cast<cudaStream_t>(stream));
 }
 
 int fp8bw_quantize_colwise(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* q_t,
@@ -264,10 +305,8 @@ int fp8bw_quantize_colwise(const uint16_t* x, int64_t rows, int64_t cols, uint8_
   if (st != FP8BW_OK) return st;
   if (rows == 0 || cols == 0) return FP8BW_OK;
   const int mode = q_row ? kModeRowCol : kModeCol;
-  return launch_quantize(mode, x, rows, cols, q_row, s_row, q_t, s_t, nullptr,
-                         static_cast<cudaStream_t>(stream)) == cudaSuccess
-             ? FP8BW_OK
-             : FP8BW_ERR_LAUNCH;
+  return launch_quantize(mode, x, rows, cols, q_row, s_row, q_t, s_t, nullptr, dev.sm_count,
+                         static_cast<cudaStream_t>(stream));
 }
 
 int fp8bw_quantize_weight_block(const uint16_t* w, int64_t n, int64_t k, uint8_t* q, float* s,
@@ -284,10 +323,8 @@ int fp8bw_quantize_weight_block(const uint16_t* w, int64_t n, int64_t k, uint8_t
   int st = current_device_info(&dev);
   if (st != FP8BW_OK) return st;
   if (n == 0 || k == 0) return FP8BW_OK;
-  return launch_quantize(kModeBlock, w, n, k, q, nullptr, q_t, nullptr, s,
-                         static_cast<cudaStream_t>(stream)) == cudaSuccess
-             ? FP8BW_OK
-             : FP8BW_ERR_LAUNCH;
+  return launch_quantize(kModeBlock, w, n, k, q, nullptr, q_t, nullptr, s, dev.sm_count,
+                         static_cast<cudaStream_t>(stream));
 }
 
 int fp8bw_gemm_fprop(const uint8_t* qx, const float* sx, const uint8_t* qw, const float* sw,

@@ -1,38 +1,53 @@
-// gemm.cuh -- blockwise-scaled E4M3 GEMM for sm_100a (tcgen05 + TMEM + TMA).
+// gemm_pair.cuh -- blockwise-scaled E4M3 GEMM for sm_100a on CTA pairs
+// (tcgen05.mma.cta_group::2 + TMEM + TMA).
 //
-// Computes, for an output tile of 128 rows x BN columns,
+// Computes, for every output element,
 //   out[i][j] = bf16( sum_c sa[c][i] * sb(c, j) * P_c[i][j] ),
 //   P_c[i][j] = sum_{kk in chunk c} A[i][kk] * B[j][kk]     (E4M3 products)
 // where c runs over 128-long chunks of the contraction dimension and sb(c, j)
-// is either one scale per 128 output columns ("block", the 128x128 weight
-// blocks of fprop and dgrad) or one per output column ("vector", the 128x1
-// token groups of wgrad). This is the per-chunk rescaling of the blockwise FP8
-// linear in the Puro-2B report (arxiv-wiki summary, "Approach" item (4); the
-// three GEMMs of paperlayer.ai summary, Appendix C, "FP8 implementation
-// pipeline"); the 128-chunk promotion interval is this library's reading.
+// is either one scale per 128 output columns ("block": the 128x128 weight
+// blocks of fprop and dgrad) or one per output column ("vector": the 128x1
+// token groups of wgrad). This is the per-chunk rescaling of the blockwise
+// FP8 linear of the Puro-2B report (arxiv-wiki summary, "Approach" item (4):
+// E4M3 with 1x128 activation groups and 128x128 weight blocks; paperlayer.ai
+// summary, Appendix C, "FP8 implementation pipeline": the forward,
+// data-gradient and weight-gradient GEMMs); fp32 accumulation with the
+// rescale at every 128-chunk is this library's reading.
 //
-// Design (one persistent CTA per SM, 384 threads, warp-specialised):
-//   warp 0      TMA producer: one 128x128 A chunk and one BNx128 B chunk per
-//               stage into a 4-stage shared-memory ring (128-byte swizzle).
-//   warp 1      allocates TMEM (2 x BN fp32 columns) and issues the MMAs: 4 x
-//               tcgen05.mma kind::f8f6f4 (M=128, N=BN, K=32) per chunk into a
-//               fresh TMEM buffer, ping-ponging two buffers, then commits the
-//               smem stage (free) and the TMEM buffer (full).
+// Output tiles of 256 rows x BN columns are computed by a cluster of two CTAs
+// on two SMs:
+//   * CTA r (r = 0, 1) holds rows [128r, 128r+128) of each A chunk and rows
+//     [r*BN/2, (r+1)*BN/2) of each B chunk (its half of N) in its shared
+//     memory; the MMA (M = 256, N = BN, K = 32, E4M3 x E4M3 -> fp32) is issued
+//     by one thread of the even CTA ("leader") and reads both CTAs' operands;
+//     each CTA's TMEM receives its own 128 rows x BN columns;
+//   * both CTAs' TMA loads count their bytes on the leader's "full" barrier
+//     (cta_group::2 TMA; no load uses cluster multicast); the leader's commits
+//     arrive on the "empty" and "TMEM full" barriers of both CTAs (multicast
+//     commit); every promotion warp of both CTAs releases a TMEM buffer on the
+//     leader's "TMEM empty" barrier;
+//   * each chunk's product goes to a fresh TMEM buffer (512 / BN buffers,
+//     round robin), so the tensor cores run ahead of the promotion.
+// Each CTA has 384 threads:
+//   warp 0      TMA producer (A and B chunks into a shared-memory ring, 128-byte
+//               swizzle)
+//   warp 1      TMEM allocation (both CTAs) and MMA issue (leader only)
 //   warp 2      scale producer: bulk-copies the chunk's 128 A-scales (and, in
-//               vector mode, BN B-scales) into an 8-slot ring; in block mode it
-//               writes the chunk's two block scales itself.
-//   warps 4-11  promotion / epilogue: warp w reads TMEM lanes 32*(w%4)..+31
-//               (its 32 output rows) and one half of the BN columns; per chunk
-//               it loads the partial sums with tcgen05.ld, hands the TMEM
-//               buffer back, and adds them, times the two scales, into an fp32
-//               accumulator held in registers (BN/2 per thread, packed f32x2
-//               FMAs); after the last chunk it converts to bf16, stages 32x32
-//               boxes in shared memory and writes them with TMA stores.
-// Registers: warps 0-3 drop to 40 per thread, the eight epilogue warps rise to
-// 232 (setmaxnreg); 4*32*40 + 8*32*232 = 384 * 168, the launch budget.
-// Every mbarrier wait is bounded (about 2 s, see common.cuh); on expiry the
-// CTA records the error, drains its outstanding copies and MMAs, frees TMEM
-// and exits.
+//               vector mode, the BN B-scales) into an 8-slot ring; in block
+//               mode it writes the chunk's block scales itself
+//   warps 4-11  promotion and epilogue: warp w reads TMEM lanes 32*(w%4)..+31
+//               (its 32 rows) and one half of the BN columns; per chunk it
+//               loads the partial sums with tcgen05.ld, hands the buffer back,
+//               and adds them, times the two scales, into fp32 accumulators
+//               held in registers (BN/2 per thread; packed f32x2 arithmetic);
+//               after the last chunk it converts to bf16, stages 32x32 boxes
+//               in shared memory and writes them with TMA stores.
+// With BN = 256 the producer warps give registers to the promotion warps
+// (setmaxnreg 56 / 224: 4*32*56 + 8*32*224 = 384 * 168, the launch budget).
+// Every mbarrier wait is bounded (about 2 s, common.cuh); on expiry the CTA
+// records the error, drains its outstanding copies and MMAs, and both CTAs
+// meet at a cluster barrier before TMEM is freed, so neither leaves while the
+// other may still touch its memory.
 #pragma once
 
 #include <cuda.h>
@@ -50,38 +65,13 @@ constexpr int kScaleStages = 8;   // scale ring depth
 constexpr int kThreads = 384;
 constexpr int kFirstEpiWarp = 4;
 constexpr int kNumEpiWarps = 8;
-constexpr int kProducerRegs = 40;
-constexpr int kEpilogueRegs = 232;
-constexpr int kLaunchRegs = 168;  // (4*32*40 + 8*32*232) / 384
+constexpr int kProducerRegs = 56;
+constexpr int kEpilogueRegs = 224;
+constexpr int kLaunchRegs = 168;  // (4*32*56 + 8*32*224) / 384
 
 static_assert(4 * 32 * kProducerRegs + kNumEpiWarps * 32 * kEpilogueRegs ==
                   kThreads * kLaunchRegs,
               "setmaxnreg split must equal the launch register budget");
-
-template <int BN, bool VEC_B>
-struct Layout {
-  static constexpr int kABytes = BM * BK;
-  static constexpr int kBBytes = BN * BK;
-  static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kRingBytes = kStages * kStageBytes;
-  static constexpr int kSaBytes = BM * 4;
-  static constexpr int kSbBytes = VEC_B ? BN * 4 : 16;
-  static constexpr int kScaleSlot = kSaBytes + kSbBytes;
-  static constexpr int kScaleOff = kRingBytes;
-  static constexpr int kBarOff = kScaleOff + kScaleStages * kScaleSlot;
-  // full[S], empty[S], sfull[SS], sempty[SS], tfull[2], tempty[2], drain
-  static constexpr int kNumBars = 2 * kStages + 2 * kScaleStages + 5;
-  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  // per epilogue warp: a 32 x 32 bf16 box (2 KB, 64-byte swizzle) staged for
-  // the TMA store of the output
-  static constexpr int kOutWarpBytes = 32 * 32 * 2;
-  static constexpr int kOutOff = ((kMiscOff + 16 + 1023) / 1024) * 1024;
-  static constexpr int kBytes = kOutOff + kNumEpiWarps * kOutWarpBytes;
-  static constexpr int kAlloc = kBytes + 1024;  // base is aligned up to 1024
-  static constexpr uint32_t kTmemCols = 2 * BN;  // power of two for BN = 128/256
-  static_assert(kBarOff % 8 == 0, "barrier alignment");
-  static_assert(kAlloc <= 227 * 1024, "shared memory budget");
-};
 
 struct Args {
   int mo, no, kc;             // output rows, output columns, contraction length
@@ -105,15 +95,44 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-template <int BN, bool VEC_B, bool B_MN>
-__global__ void __launch_bounds__(kThreads, 1)
-    blockwise_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
-                          const __grid_constant__ CUtensorMap tm_b,
-                          const __grid_constant__ CUtensorMap tm_out,
-                          const Args g) {
-  using L = Layout<BN, VEC_B>;
+
+template <int BN_, bool VEC_B>
+struct PairLayout {
+  static constexpr int BN = BN_;                 // pair tile columns (128 or 256)
+  static constexpr int kStages = BN == 256 ? 6 : 8;
+  static constexpr int kTmemBufs = 512 / BN;     // fp32 partial buffers in TMEM
+  static constexpr int kABytes = BM * BK;        // this CTA's 128 A rows
+  static constexpr int kBBytes = (BN / 2) * BK;  // this CTA's BN/2 B rows
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kRingBytes = kStages * kStageBytes;
+  static constexpr int kSaBytes = BM * 4;
+  static constexpr int kSbBytes = VEC_B ? BN * 4 : 16;
+  static constexpr int kScaleSlot = kSaBytes + kSbBytes;
+  static constexpr int kScaleOff = kRingBytes;
+  static constexpr int kBarOff = kScaleOff + kScaleStages * kScaleSlot;
+  static constexpr int kNumBars = 2 * kStages + 2 * kScaleStages + 2 * kTmemBufs + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kOutWarpBytes = 32 * 32 * 2;
+  static constexpr int kOutOff = ((kMiscOff + 16 + 1023) / 1024) * 1024;
+  static constexpr int kBytes = kOutOff + kNumEpiWarps * kOutWarpBytes;
+  static constexpr int kAlloc = kBytes + 1024;
+  static constexpr uint32_t kTmemCols = 512;     // kTmemBufs x BN columns
+  static_assert(kAlloc <= 227 * 1024, "shared memory budget");
+};
+
+template <int BN_, bool VEC_B, bool B_MN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    blockwise_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
+                               const __grid_constant__ CUtensorMap tm_b,
+                               const __grid_constant__ CUtensorMap tm_out,
+                               const Args g) {
+  using L = PairLayout<BN_, VEC_B>;
+  constexpr int BN = L::BN;
+  constexpr int kPairStages = L::kStages;
+  constexpr int kBufs = L::kTmemBufs;
+  static_assert(!B_MN || BN == 256, "MN-major B uses full 128-element swizzle atoms");
   constexpr int kHalf = BN / 2;                      // columns per epilogue thread
-  constexpr uint32_t kIdesc = idesc_e4m3(BM, BN, B_MN);
+  constexpr uint32_t kIdesc = idesc_e4m3(2 * BM, BN, B_MN);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -121,30 +140,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + L::kBarOff;
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
-  auto sfull_bar = [&](int s) { return bar0 + 8u * (2 * kStages + s); };
-  auto sempty_bar = [&](int s) { return bar0 + 8u * (2 * kStages + kScaleStages + s); };
-  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * kStages + 2 * kScaleStages + b); };
-  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * kStages + 2 * kScaleStages + 2 + b); };
-  const uint32_t drain_bar = bar0 + 8u * (2 * kStages + 2 * kScaleStages + 4);
+  auto empty_bar = [&](int s) { return bar0 + 8u * (kPairStages + s); };
+  auto sfull_bar = [&](int s) { return bar0 + 8u * (2 * kPairStages + s); };
+  auto sempty_bar = [&](int s) { return bar0 + 8u * (2 * kPairStages + kScaleStages + s); };
+  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * kPairStages + 2 * kScaleStages + b); };
+  auto tempty_bar = [&](int b) {
+    return bar0 + 8u * (2 * kPairStages + 2 * kScaleStages + kBufs + b);
+  };
+  const uint32_t drain_bar = bar0 + 8u * (2 * kPairStages + 2 * kScaleStages + 2 * kBufs);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L::kMiscOff);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();           // 0 = leader, 1 = follower
+  const bool leader = rank == 0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
+    for (int s = 0; s < kPairStages; ++s) {
+      mbar_init(full_bar(s), 1);      // leader: its own expect_tx arrival
+      mbar_init(empty_bar(s), 1);     // one multicast commit
     }
     for (int s = 0; s < kScaleStages; ++s) {
       mbar_init(sfull_bar(s), 1);
       mbar_init(sempty_bar(s), kNumEpiWarps);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kBufs; ++b) {
       mbar_init(tfull_bar(b), 1);
-      mbar_init(tempty_bar(b), kNumEpiWarps);
+      mbar_init(tempty_bar(b), 2 * kNumEpiWarps);  // used on the leader only
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0u;
@@ -156,71 +179,77 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tm_out);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), L::kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(smem_u32(const_cast<uint32_t*>(tmem_slot)), L::kTmemCols);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  // Barrier initialisation and TMEM allocation visible to both CTAs.
+  cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int num_tiles = g.tiles_m * g.tiles_n;
+  const int num_tiles = g.tiles_m * g.tiles_n;       // pair tiles (256 x 256)
   const int C = g.chunks;
+  const int cluster_id = blockIdx.x >> 1;
+  const int num_clusters = gridDim.x >> 1;
 
-  if (warp < kFirstEpiWarp) setmaxnreg_dec();
+  // BN = 256: the promotion warps hold 128 accumulators + 64 loaded partials
+  // per thread, so registers move from the producer warps to them. BN = 128
+  // fits the launch allocation as it is.
+  if constexpr (BN == 256) {
+    if (warp < kFirstEpiWarp) setmaxnreg_dec();
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      const uint32_t full_leader0 = mapa_shared(full_bar(0), 0);
       uint32_t it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+      for (int tile = cluster_id; ok && tile < num_tiles; tile += num_clusters) {
         const int tm = tile / g.tiles_n, tn = tile % g.tiles_n;
+        const int a_row = tm * (2 * BM) + static_cast<int>(rank) * BM;
+        const int b_row = tn * BN + static_cast<int>(rank) * (BN / 2);
         for (int c = 0; c < C; ++c, ++it) {
-          const int s = it % kStages;
-          const uint32_t u = it / kStages;
+          const int s = it % kPairStages;
+          const uint32_t u = it / kPairStages;
           if (!mbar_wait(empty_bar(s), (u & 1u) ^ 1u, abort_flag, kErrTimeoutTma)) {
             ok = false;
             break;
           }
           const uint32_t a_dst = sbase + s * L::kStageBytes;
           const uint32_t b_dst = a_dst + L::kABytes;
-          mbar_arrive_expect_tx(full_bar(s), L::kStageBytes);
-          tma_load_2d(a_dst, &tm_a, full_bar(s), c * BK, tm * BM);
-          if constexpr (B_MN) {
-#pragma unroll
-            for (int h = 0; h < BN / 128; ++h)
-              tma_load_2d(b_dst + h * 128 * BK, &tm_b, full_bar(s),
-                          tn * BN + h * 128, c * BK);
-          } else {
-            tma_load_2d(b_dst, &tm_b, full_bar(s), c * BK, tn * BN);
-          }
+          const uint32_t fbar = full_leader0 + 8u * s;
+          if (leader) mbar_arrive_expect_tx(full_bar(s), 2 * L::kStageBytes);
+          tma_load_2d_pair(a_dst, &tm_a, fbar, c * BK, a_row);
+          if constexpr (B_MN)
+            tma_load_2d_pair(b_dst, &tm_b, fbar, b_row, c * BK);
+          else
+            tma_load_2d_pair(b_dst, &tm_b, fbar, c * BK, b_row);
         }
       }
-      if (!ok) {
-        // Drain: every stage filled in the last kStages iterations must land
-        // before the CTA's shared memory is released.
-        for (uint32_t k = 0; k < kStages && k < it; ++k) {
+      if (!ok && leader) {
+        for (uint32_t k = 0; k < kPairStages && k < it; ++k) {
           const uint32_t j = it - 1 - k;
-          const uint32_t ph = (j / kStages) & 1u;
+          const uint32_t ph = (j / kPairStages) & 1u;
           const uint64_t t0 = globaltimer_ns();
-          while (!mbar_try_wait(full_bar(j % kStages), ph) &&
+          while (!mbar_try_wait(full_bar(j % kPairStages), ph) &&
                  globaltimer_ns() - t0 < kWaitLimitNs) {
           }
         }
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (leader && lane == 0) {
       uint32_t it = 0, tc = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+      for (int tile = cluster_id; ok && tile < num_tiles; tile += num_clusters) {
         for (int c = 0; c < C; ++c, ++it, ++tc) {
-          const int s = it % kStages;
-          const uint32_t u = it / kStages;
-          const int tb = tc & 1;
-          const uint32_t tu = tc >> 1;
+          const int s = it % kPairStages;
+          const uint32_t u = it / kPairStages;
+          const int tb = tc % kBufs;
+          const uint32_t tu = tc / kBufs;
           if (!mbar_wait(full_bar(s), u & 1u, abort_flag, kErrTimeoutMma) ||
               !mbar_wait(tempty_bar(tb), (tu & 1u) ^ 1u, abort_flag, kErrTimeoutMma)) {
             ok = false;
@@ -238,15 +267,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               bdesc = desc_mnmajor_sw128(b_addr + kk * 32 * 128, 128 * BK);
             else
               bdesc = desc_kmajor_sw128(b_addr + kk * 32);
-            mma_f8(d_tmem, adesc, bdesc, kIdesc, kk > 0 ? 1u : 0u);
+            mma_f8_pair(d_tmem, adesc, bdesc, kIdesc, kk > 0 ? 1u : 0u);
           }
-          mma_commit(empty_bar(s));
-          mma_commit(tfull_bar(tb));
+          mma_commit_pair(empty_bar(s), 0x3);
+          mma_commit_pair(tfull_bar(tb), 0x3);
         }
       }
       if (!ok) {
-        // Drain the MMAs already issued before TMEM is released.
-        mma_commit(drain_bar);
+        mma_commit_pair(drain_bar, 0x1);
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(drain_bar, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
         }
@@ -256,17 +284,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ scale producer
     uint32_t sit = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+    for (int tile = cluster_id; ok && tile < num_tiles; tile += num_clusters) {
       const int tm = tile / g.tiles_n, tn = tile % g.tiles_n;
-      const int m0 = tm * BM, n0 = tn * BN;
-      const uint32_t a_bytes = static_cast<uint32_t>(min(BM, g.mo - m0)) * 4u;
+      const int m0 = tm * (2 * BM) + static_cast<int>(rank) * BM, n0 = tn * BN;
+      const int rows_here = max(0, min(BM, g.mo - m0));
+      const uint32_t a_bytes = static_cast<uint32_t>(rows_here) * 4u;
       const uint32_t b_bytes = VEC_B ? static_cast<uint32_t>(min(BN, g.no - n0)) * 4u : 0u;
       const int jb0 = n0 / 128;
       float pre0 = 0.0f, pre1 = 0.0f;
       for (int c = 0; c < C; ++c, ++sit) {
         if constexpr (!VEC_B) {
           if ((c & 31) == 0) {
-            // lane l fetches the block scales of chunk c + l (both blocks)
             const int cc = c + lane;
             pre0 = 0.0f;
             pre1 = 0.0f;
@@ -292,8 +320,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               reinterpret_cast<float*>(slot + L::kSaBytes)[1] = v1;
             }
             mbar_arrive_expect_tx(sfull_bar(ss), a_bytes + b_bytes);
-            bulk_load(slot_u, g.sa + static_cast<int64_t>(c) * g.mo + m0, a_bytes,
-                      sfull_bar(ss));
+            if (a_bytes > 0)
+              bulk_load(slot_u, g.sa + static_cast<int64_t>(c) * g.mo + m0, a_bytes,
+                        sfull_bar(ss));
             if constexpr (VEC_B)
               bulk_load(slot_u + L::kSaBytes, g.sb + static_cast<int64_t>(c) * g.no + n0,
                         b_bytes, sfull_bar(ss));
@@ -318,23 +347,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kFirstEpiWarp) {
     // ------------------------------------------------------------ promotion + epilogue
-    setmaxnreg_inc();
+    if constexpr (BN == 256) setmaxnreg_inc();
     const int q = warp & 3;                          // TMEM lane quarter
     const int ew = warp - kFirstEpiWarp;
     const int h = ew >> 2;                           // column half of the tile
-    const int row = q * 32 + lane;                   // tile row = TMEM lane
+    const int row = q * 32 + lane;                   // this CTA's tile row = TMEM lane
     const uint32_t stage_out = sbase + L::kOutOff + ew * L::kOutWarpBytes;
+    const uint32_t tempty_leader0 = mapa_shared(tempty_bar(0), 0);
     uint32_t tc = 0, sit = 0;
     bool ok = true, store_pending = false;
-    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+    for (int tile = cluster_id; ok && tile < num_tiles; tile += num_clusters) {
       const int tm = tile / g.tiles_n, tn = tile % g.tiles_n;
       float acc[kHalf];
 #pragma unroll
       for (int j = 0; j < kHalf; ++j) acc[j] = 0.0f;
 
       for (int c = 0; c < C; ++c, ++tc, ++sit) {
-        const int tb = tc & 1;
-        const uint32_t tu = tc >> 1;
+        const int tb = tc % kBufs;
+        const uint32_t tu = tc / kBufs;
         const int ss = sit % kScaleStages;
         const uint32_t su = sit / kScaleStages;
         if (!mbar_wait(tfull_bar(tb), tu & 1u, abort_flag, kErrTimeoutEpi) ||
@@ -345,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const float* slot = reinterpret_cast<const float*>(smem + L::kScaleOff + ss * L::kScaleSlot);
         const float sa_v = slot[row];
-        const float* sbv = slot + BM;                 // B scales of this chunk
+        const float* sbv = slot + BM;
         float blk_scale = 0.0f;
         if constexpr (!VEC_B) blk_scale = sa_v * sbv[BN > 128 ? h : 0];
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
@@ -357,11 +387,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(taddr + part * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
           tmem_wait_ld();
           if (part == kHalf / 64 - 1) {
-            // Every TMEM read of this chunk has landed: hand the buffer back to
-            // the MMA warp before doing the arithmetic.
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(tempty_bar(tb));
+            if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8u * tb);
           }
           float* a = acc + part * 64;
           if constexpr (VEC_B) {
@@ -387,10 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
 
-      // ---- bf16 output through shared memory and TMA stores: this warp owns
-      // rows [m0 + 32q, +32) and columns [n0 + h*kHalf, +kHalf), written as
-      // 32 x 32 boxes (64-byte rows, 16-byte chunks xor-swizzled by row/2).
-      const int y0 = tm * BM + q * 32;
+      const int y0 = tm * (2 * BM) + static_cast<int>(rank) * BM + q * 32;
       const int x0 = tn * BN + h * kHalf;
 #pragma unroll
       for (int gi = 0; gi < kHalf / 32; ++gi) {
@@ -424,10 +449,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  // Neither CTA frees TMEM or leaves while its pair may still read its shared
+  // memory, write its TMEM or arrive on its barriers.
+  cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, L::kTmemCols);
+    tmem_dealloc_pair(tmem_base, L::kTmemCols);
   }
 }
 

@@ -6,20 +6,31 @@
 // qscale = 448/amax, s = amax/448 (fp32, round-to-nearest-even), amax == 0 or
 // an overflowing qscale gives qscale = s = 1; code = E4M3_satfinite_rn(x*qscale).
 //
-// One CTA of 256 threads owns a 128x128 tile of the bf16 input (32 KB).
-// Thread t holds an 8x8 sub-block: rows 8*(t/16) .. +7, columns 8*(t%16) .. +7,
-// read as eight 16-byte vectors (each warp instruction reads two full 256-byte
-// row segments). From the registers it derives
+// One persistent kernel, several modes. Each CTA (256 threads, two per SM)
+// walks 128x128 tiles of the bf16 input; the next two tiles are fetched by TMA
+// into a double-buffered shared-memory ring while the current one is worked
+// on, so HBM reads stay in flight across the whole kernel.
+// Thread t owns an 8x8 sub-block of the tile: rows 8*(t/16) .. +7, columns
+// 8*(t%16) .. +7, read from shared memory as eight 16-byte vectors. From the
+// registers it derives
 //   * row groups (1x128): the 16 threads of a half-warp share a row, so the
-//     amax is a 4-step xor shuffle;
-//   * column groups (128x1): per-thread max over its 8 rows, a shuffle with the
-//     other half-warp, then a 8-warp reduction through shared memory;
-//   * the 128x128 block amax: a warp reduction plus the same 8-warp step.
-// Row codes go out as 8-byte stores (16 lanes cover a 128-byte row segment);
-// transposed codes as 8-byte stores of 8 consecutive tokens of one column.
-// Nothing is staged through global memory; scratch is 4.5 KB of shared memory.
+//     amax is a 4-step xor shuffle; codes leave as 8-byte stores (a half-warp
+//     writes one 128-byte row segment), scales through shared memory as one
+//     512-byte run;
+//   * column groups (128x1): per-thread max over its 8 rows, a shuffle with
+//     the other half-warp, then an 8-warp reduction through shared memory; the
+//     transposed codes (8 tokens of one column = 8 bytes per thread) go to a
+//     128x128-byte shared tile, 8-byte units xor-swizzled by column block so
+//     the writes are bank-conflict free, and leave as coalesced 16-byte rows;
+//   * the 128x128 block amax (weights): a warp reduction plus the 8-warp step.
+// Shared memory per CTA: 64 KB input ring + 16 KB transposed codes + 5 KB.
+#pragma once
+
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
+
+#include <mutex>
 
 #include "common.cuh"
 
@@ -27,24 +38,38 @@ namespace fp8bw {
 
 namespace {
 
-constexpr int kTile = 128;
-constexpr int kThreads = 256;
+constexpr int kQTile = 128;
+constexpr int kQThreads = 256;
+constexpr int kQTileBytes = kQTile * kQTile * 2;  // one bf16 input tile
 
 enum QuantMode : int {
-  kModeRow = 0,    // row-wise codes + scales
-  kModeCol = 1,    // transposed column-wise codes + scales
-  kModeRowCol = 2, // both, one read of the input
-  kModeBlock = 3,  // 128x128 block scale; codes row-major and optionally transposed
+  kModeRow = 0,     // row-wise codes + scales
+  kModeCol = 1,     // transposed column-wise codes + scales
+  kModeRowCol = 2,  // both, one read of the input
+  kModeBlock = 3,   // 128x128 block scale; codes row-major and optionally transposed
 };
 
 struct QuantArgs {
-  const uint16_t* x;
   int64_t rows, cols;
+  int tiles_r, tiles_c;
   uint8_t* q_row;   // [rows, cols]  (block mode: q)
   float* s_row;     // [ceil(cols/128)][rows]
   uint8_t* q_col;   // [cols, rows]  (block mode: q_t, may be null)
   float* s_col;     // [ceil(rows/128)][cols]
   float* s_block;   // [ceil(rows/128)][ceil(cols/128)]
+};
+
+struct QuantSmem {
+  static constexpr int kIn = 0;                                 // 2 x 32 KB
+  static constexpr int kT = 2 * kQTileBytes;                    // 16 KB
+  static constexpr int kRed = kT + kQTile * kQTile;             // 8 x 128 floats
+  static constexpr int kColQ = kRed + 8 * kQTile * 4;           // 128 floats
+  static constexpr int kSRow = kColQ + kQTile * 4;              // 128 floats
+  static constexpr int kBlk = kSRow + kQTile * 4;               // 8 floats
+  static constexpr int kBar = kBlk + 64;                        // 2 mbarriers
+  static constexpr int kFlag = kBar + 16;
+  static constexpr int kBytes = kFlag + 16;
+  static constexpr int kAlloc = kBytes + 128;                   // base aligned to 128
 };
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) {
@@ -82,70 +107,127 @@ __device__ __forceinline__ uint2 pack8(const float (&t)[8]) {
   return r;
 }
 
+// Byte offset, in the transposed tile T[col][token], of the 8-byte unit that
+// holds tokens 8*u .. 8*u+7 of column k: the unit index is xor-ed with the
+// column block k/8, so the 16 column blocks of a half-warp hit 16 different
+// bank pairs.
+__device__ __forceinline__ int t_unit_offset(int k, int u) {
+  return k * kQTile + ((u ^ (k >> 3)) & 15) * 8;
+}
+
 template <int MODE>
-__global__ void __launch_bounds__(kThreads) quant_tile_kernel(QuantArgs a) {
-  __shared__ __align__(16) float red[kThreads / 32][kTile];  // per-warp column maxima
-  __shared__ __align__(16) float colq[kTile];                // column qscales
-  __shared__ float blk[kThreads / 32];
+__global__ void __launch_bounds__(kQThreads, 2)
+    quant_tile_kernel(const __grid_constant__ CUtensorMap tm_x, const QuantArgs a) {
+  extern __shared__ uint8_t qsmem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(qsmem_raw) + 127) & ~static_cast<uintptr_t>(127));
+  using S = QuantSmem;
+  float(*red)[kQTile] = reinterpret_cast<float(*)[kQTile]>(smem + S::kRed);
+  float* colq = reinterpret_cast<float*>(smem + S::kColQ);
+  float* srow_s = reinterpret_cast<float*>(smem + S::kSRow);
+  float* blk = reinterpret_cast<float*>(smem + S::kBlk);
+  uint8_t* T = smem + S::kT;
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + S::kBar;
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + S::kFlag);
 
   const int t = threadIdx.x;
   const int warp = t >> 5;
   const int lane = t & 31;
   const int rb = t >> 4;   // 0..15: rows 8*rb .. 8*rb+7 of the tile
   const int cg = t & 15;   // 0..15: columns 8*cg .. 8*cg+7 of the tile
-
   const int64_t rows = a.rows, cols = a.cols;
-  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * kTile + rb * 8;
-  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kTile + cg * 8;
-  // rows and cols are multiples of 16: an 8-wide run is all in or all out.
-  const bool cvalid = c0 < cols;
-  const bool rvalid = r0 < rows;
+  const int num_tiles = a.tiles_r * a.tiles_c;
 
-  // ---- load the 8x8 sub-block as packed bf16 pairs (zeros outside) --------
-  uint32_t v[8][4];
-#pragma unroll
-  for (int p = 0; p < 8; ++p) {
-    uint4 w = make_uint4(0u, 0u, 0u, 0u);
-    if (cvalid && rvalid)
-      w = __ldcs(reinterpret_cast<const uint4*>(a.x + (r0 + p) * cols + c0));
-    v[p][0] = w.x;
-    v[p][1] = w.y;
-    v[p][2] = w.z;
-    v[p][3] = w.w;
+  if (t == 0) {
+    mbar_init(bar0, 1);
+    mbar_init(bar0 + 8, 1);
+    *abort_flag = 0u;
+    fence_mbar_init();
+    prefetch_tmap(&tm_x);
+  }
+  __syncthreads();
+  // Thread 0 keeps, per input buffer, the phase parity of a load it issued and
+  // that nobody has waited for yet (-1: none).
+  int pend[2] = {-1, -1};
+  if (t == 0) {
+    for (int k = 0; k < 2; ++k) {
+      const int tile = blockIdx.x + k * gridDim.x;
+      if (tile < num_tiles) {
+        mbar_arrive_expect_tx(bar0 + 8u * k, kQTileBytes);
+        tma_load_2d(sbase + S::kIn + k * kQTileBytes, &tm_x, bar0 + 8u * k,
+                    (tile % a.tiles_c) * kQTile, (tile / a.tiles_c) * kQTile);
+        pend[k] = 0;
+      }
+    }
   }
 
-  if constexpr (MODE == kModeBlock) {
-    // ---- one amax for the whole 128x128 block ------------------------------
-    float m = 0.0f;
-#pragma unroll
-    for (int p = 0; p < 8; ++p)
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        m = fmaxf(m, fmaxf(fabsf(bf16_lo(v[p][j])), fabsf(bf16_hi(v[p][j]))));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    if (lane == 0) blk[warp] = m;
-    __syncthreads();
-    float amax = blk[0];
-#pragma unroll
-    for (int w = 1; w < kThreads / 32; ++w) amax = fmaxf(amax, blk[w]);
-    float qs, s;
-    group_scale(amax, qs, s);
-    if (t == 0) {
-      const int64_t nkb = (cols + kTile - 1) / kTile;
-      a.s_block[static_cast<int64_t>(blockIdx.y) * nkb + blockIdx.x] = s;
-    }
-    if (cvalid && rvalid) {
+  int k = 0;
+  for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++k) {
+    const int buf = k & 1;
+    const bool got = mbar_wait(bar0 + 8u * buf, (k >> 1) & 1, abort_flag, kErrTimeoutTma);
+    if (!__syncthreads_and(got ? 1 : 0)) break;
+    pend[buf] = -1;
+    const int tr = tile / a.tiles_c, tc = tile % a.tiles_c;
+    const int64_t r0 = static_cast<int64_t>(tr) * kQTile + rb * 8;
+    const int64_t c0 = static_cast<int64_t>(tc) * kQTile + cg * 8;
+    // rows and cols are multiples of 16: an 8-wide run is all in or all out.
+    const bool cvalid = c0 < cols;
+    const bool rvalid = r0 < rows;
+
+    // ---- the 8x8 sub-block from shared memory (zeros outside the tensor) --
+    uint32_t v[8][4];
+    {
+      const uint16_t* in = reinterpret_cast<const uint16_t*>(smem + S::kIn + buf * kQTileBytes);
 #pragma unroll
       for (int p = 0; p < 8; ++p) {
-        float tv[8];
+        const uint4 w = *reinterpret_cast<const uint4*>(in + (rb * 8 + p) * kQTile + cg * 8);
+        v[p][0] = w.x;
+        v[p][1] = w.y;
+        v[p][2] = w.z;
+        v[p][3] = w.w;
+      }
+    }
+    __syncthreads();  // the input buffer is free: fetch the tile after next
+    if (t == 0) {
+      const int next = tile + 2 * gridDim.x;
+      if (next < num_tiles) {
+        mbar_arrive_expect_tx(bar0 + 8u * buf, kQTileBytes);
+        tma_load_2d(sbase + S::kIn + buf * kQTileBytes, &tm_x, bar0 + 8u * buf,
+                    (next % a.tiles_c) * kQTile, (next / a.tiles_c) * kQTile);
+        pend[buf] = ((k >> 1) + 1) & 1;
+      }
+    }
+
+    if constexpr (MODE == kModeBlock) {
+      // ---- one amax for the whole 128x128 block -----------------------------
+      float m = 0.0f;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          tv[2 * j] = __fmul_rn(bf16_lo(v[p][j]), qs);
-          tv[2 * j + 1] = __fmul_rn(bf16_hi(v[p][j]), qs);
+      for (int p = 0; p < 8; ++p)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          m = fmaxf(m, fmaxf(fabsf(bf16_lo(v[p][j])), fabsf(bf16_hi(v[p][j]))));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+      if (lane == 0) blk[warp] = m;
+      __syncthreads();
+      float amax = blk[0];
+#pragma unroll
+      for (int w = 1; w < kQThreads / 32; ++w) amax = fmaxf(amax, blk[w]);
+      float qs, s;
+      group_scale(amax, qs, s);
+      if (t == 0) a.s_block[static_cast<int64_t>(tr) * a.tiles_c + tc] = s;
+      if (cvalid && rvalid) {
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+          float tv[8];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            tv[2 * j] = __fmul_rn(bf16_lo(v[p][j]), qs);
+            tv[2 * j + 1] = __fmul_rn(bf16_hi(v[p][j]), qs);
+          }
+          *reinterpret_cast<uint2*>(a.q_row + (r0 + p) * cols + c0) = pack8(tv);
         }
-        *reinterpret_cast<uint2*>(a.q_row + (r0 + p) * cols + c0) = pack8(tv);
       }
       if (a.q_col != nullptr) {
 #pragma unroll
@@ -156,82 +238,68 @@ __global__ void __launch_bounds__(kThreads) quant_tile_kernel(QuantArgs a) {
             const float x = (j & 1) ? bf16_hi(v[p][j >> 1]) : bf16_lo(v[p][j >> 1]);
             tv[p] = __fmul_rn(x, qs);
           }
-          *reinterpret_cast<uint2*>(a.q_col + (c0 + j) * rows + r0) = pack8(tv);
+          *reinterpret_cast<uint2*>(T + t_unit_offset(cg * 8 + j, rb)) = pack8(tv);
         }
       }
-    }
-    return;
-  } else {
-    if constexpr (MODE == kModeRow || MODE == kModeRowCol) {
-      // ---- row groups: 16 lanes of a half-warp share each row --------------
-      float srow[8];
-#pragma unroll
-      for (int p = 0; p < 8; ++p) {
-        float m = 0.0f;
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          m = fmaxf(m, fmaxf(fabsf(bf16_lo(v[p][j])), fabsf(bf16_hi(v[p][j]))));
-#pragma unroll
-        for (int o = 8; o > 0; o >>= 1)
-          m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-        float qs, s;
-        group_scale(m, qs, s);
-        srow[p] = s;
-        if (cvalid && rvalid) {
-          float tv[8];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            tv[2 * j] = __fmul_rn(bf16_lo(v[p][j]), qs);
-            tv[2 * j + 1] = __fmul_rn(bf16_hi(v[p][j]), qs);
-          }
-          *reinterpret_cast<uint2*>(a.q_row + (r0 + p) * cols + c0) = pack8(tv);
-        }
-      }
-      if (cg == 0 && rvalid && blockIdx.x * kTile < cols) {
-        float* dst = a.s_row + static_cast<int64_t>(blockIdx.x) * rows + r0;
-        reinterpret_cast<float4*>(dst)[0] =
-            make_float4(srow[0], srow[1], srow[2], srow[3]);
-        reinterpret_cast<float4*>(dst)[1] =
-            make_float4(srow[4], srow[5], srow[6], srow[7]);
-      }
-    }
-
-    if constexpr (MODE == kModeCol || MODE == kModeRowCol) {
-      // ---- column groups: 8 rows here, x2 across the half-warps, x8 warps --
-      float cm[8];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        float lo = 0.0f, hi = 0.0f;
+    } else {
+      if constexpr (MODE == kModeRow || MODE == kModeRowCol) {
+        // ---- row groups: 16 lanes of a half-warp share each row ------------
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
-          lo = fmaxf(lo, fabsf(bf16_lo(v[p][j])));
-          hi = fmaxf(hi, fabsf(bf16_hi(v[p][j])));
+          float m = 0.0f;
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            m = fmaxf(m, fmaxf(fabsf(bf16_lo(v[p][j])), fabsf(bf16_hi(v[p][j]))));
+#pragma unroll
+          for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+          float qs, s;
+          group_scale(m, qs, s);
+          if (cg == 0) srow_s[rb * 8 + p] = s;
+          if (cvalid && rvalid) {
+            float tv[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              tv[2 * j] = __fmul_rn(bf16_lo(v[p][j]), qs);
+              tv[2 * j + 1] = __fmul_rn(bf16_hi(v[p][j]), qs);
+            }
+            *reinterpret_cast<uint2*>(a.q_row + (r0 + p) * cols + c0) = pack8(tv);
+          }
         }
-        cm[2 * j] = lo;
-        cm[2 * j + 1] = hi;
       }
+
+      if constexpr (MODE == kModeCol || MODE == kModeRowCol) {
+        // ---- column groups: 8 rows here, x2 across the half-warps, x8 warps
+        float cm[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        cm[j] = fmaxf(cm[j], __shfl_xor_sync(0xFFFFFFFFu, cm[j], 16));
-      if (lane < 16) {
-        float4* dst = reinterpret_cast<float4*>(&red[warp][cg * 8]);
-        dst[0] = make_float4(cm[0], cm[1], cm[2], cm[3]);
-        dst[1] = make_float4(cm[4], cm[5], cm[6], cm[7]);
-      }
-      __syncthreads();
-      if (t < kTile) {
-        float m = red[0][t];
+        for (int j = 0; j < 4; ++j) {
+          float lo = 0.0f, hi = 0.0f;
 #pragma unroll
-        for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, red[w][t]);
-        float qs, s;
-        group_scale(m, qs, s);
-        colq[t] = qs;
-        const int64_t col = static_cast<int64_t>(blockIdx.x) * kTile + t;
-        if (col < cols && static_cast<int64_t>(blockIdx.y) * kTile < rows)
-          a.s_col[static_cast<int64_t>(blockIdx.y) * cols + col] = s;
-      }
-      __syncthreads();
-      if (cvalid && rvalid) {
+          for (int p = 0; p < 8; ++p) {
+            lo = fmaxf(lo, fabsf(bf16_lo(v[p][j])));
+            hi = fmaxf(hi, fabsf(bf16_hi(v[p][j])));
+          }
+          cm[2 * j] = lo;
+          cm[2 * j + 1] = hi;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) cm[j] = fmaxf(cm[j], __shfl_xor_sync(0xFFFFFFFFu, cm[j], 16));
+        if (lane < 16) {
+          float4* dst = reinterpret_cast<float4*>(&red[warp][cg * 8]);
+          dst[0] = make_float4(cm[0], cm[1], cm[2], cm[3]);
+          dst[1] = make_float4(cm[4], cm[5], cm[6], cm[7]);
+        }
+        __syncthreads();
+        if (t < kQTile) {
+          float m = red[0][t];
+#pragma unroll
+          for (int w = 1; w < kQThreads / 32; ++w) m = fmaxf(m, red[w][t]);
+          float qs, s;
+          group_scale(m, qs, s);
+          colq[t] = qs;
+          const int64_t col = static_cast<int64_t>(tc) * kQTile + t;
+          if (col < cols) a.s_col[static_cast<int64_t>(tr) * cols + col] = s;
+        }
+        __syncthreads();
         const float4 q0 = *reinterpret_cast<const float4*>(&colq[cg * 8]);
         const float4 q1 = *reinterpret_cast<const float4*>(&colq[cg * 8 + 4]);
         const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
@@ -243,8 +311,49 @@ __global__ void __launch_bounds__(kThreads) quant_tile_kernel(QuantArgs a) {
             const float x = (j & 1) ? bf16_hi(v[p][j >> 1]) : bf16_lo(v[p][j >> 1]);
             tv[p] = __fmul_rn(x, qv[j]);
           }
-          *reinterpret_cast<uint2*>(a.q_col + (c0 + j) * rows + r0) = pack8(tv);
+          *reinterpret_cast<uint2*>(T + t_unit_offset(cg * 8 + j, rb)) = pack8(tv);
         }
+      }
+    }
+
+    __syncthreads();  // T (and the row scales) complete
+    if constexpr (MODE == kModeRow || MODE == kModeRowCol) {
+      // row scales: one 512-byte run s_row[tc][tr*128 .. +127]
+      if (t < kQTile / 4) {
+        const int64_t row = static_cast<int64_t>(tr) * kQTile + t * 4;
+        if (row < rows)
+          *reinterpret_cast<float4*>(a.s_row + static_cast<int64_t>(tc) * rows + row) =
+              *reinterpret_cast<const float4*>(&srow_s[t * 4]);
+      }
+    }
+    if (MODE == kModeCol || MODE == kModeRowCol || (MODE == kModeBlock && a.q_col != nullptr)) {
+      // transposed codes: column k of the tile is 128 contiguous tokens of
+      // q_col row (tc*128 + k); 8 threads write one 128-byte row, 16 bytes each.
+#pragma unroll
+      for (int it = 0; it < 4; ++it) {
+        const int idx = it * kQThreads + t;   // 0..1023
+        const int kk = idx >> 3;              // tile column
+        const int ch = idx & 7;               // 16-byte chunk = units 2ch, 2ch+1
+        const int64_t col = static_cast<int64_t>(tc) * kQTile + kk;
+        const int64_t tok = static_cast<int64_t>(tr) * kQTile + ch * 16;
+        if (col < cols && tok < rows) {
+          const uint2 lo = *reinterpret_cast<const uint2*>(T + t_unit_offset(kk, 2 * ch));
+          const uint2 hi = *reinterpret_cast<const uint2*>(T + t_unit_offset(kk, 2 * ch + 1));
+          *reinterpret_cast<uint4*>(a.q_col + col * rows + tok) = make_uint4(lo.x, lo.y, hi.x, hi.y);
+        }
+      }
+    }
+    __syncthreads();  // T and the scale staging may be reused
+  }
+
+  if (t == 0) {
+    // After an expired wait the loop ends early: let the copies already issued
+    // land before the shared memory is released (bounded as well).
+    for (int b = 0; b < 2; ++b) {
+      if (pend[b] < 0) continue;
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(bar0 + 8u * b, static_cast<uint32_t>(pend[b])) &&
+             globaltimer_ns() - t0 < kWaitLimitNs) {
       }
     }
   }
@@ -252,29 +361,36 @@ __global__ void __launch_bounds__(kThreads) quant_tile_kernel(QuantArgs a) {
 
 }  // namespace
 
+// 2-D bf16 tensor [rows, cols] read in 128 x 128 boxes (256-byte rows, no
+// swizzle); out-of-range elements read as zero.
+int encode_bf16_in(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows);
+
 // Launchers (shapes and pointers already validated by the C ABI layer).
-cudaError_t launch_quantize(int mode, const uint16_t* x, int64_t rows,
-                            int64_t cols, uint8_t* q_row, float* s_row,
-                            uint8_t* q_col, float* s_col, float* s_block,
-                            cudaStream_t stream) {
-  QuantArgs a{x, rows, cols, q_row, s_row, q_col, s_col, s_block};
-  dim3 grid(static_cast<unsigned>((cols + kTile - 1) / kTile),
-            static_cast<unsigned>((rows + kTile - 1) / kTile));
-  switch (mode) {
-    case kModeRow:
-      quant_tile_kernel<kModeRow><<<grid, kThreads, 0, stream>>>(a);
-      break;
-    case kModeCol:
-      quant_tile_kernel<kModeCol><<<grid, kThreads, 0, stream>>>(a);
-      break;
-    case kModeRowCol:
-      quant_tile_kernel<kModeRowCol><<<grid, kThreads, 0, stream>>>(a);
-      break;
-    default:
-      quant_tile_kernel<kModeBlock><<<grid, kThreads, 0, stream>>>(a);
-      break;
-  }
-  return cudaGetLastError();
+int launch_quantize(int mode, const uint16_t* x, int64_t rows, int64_t cols, uint8_t* q_row,
+                    float* s_row, uint8_t* q_col, float* s_col, float* s_block, int sm_count,
+                    cudaStream_t stream) {
+  QuantArgs a{rows, cols, static_cast<int>((rows + kQTile - 1) / kQTile),
+              static_cast<int>((cols + kQTile - 1) / kQTile), q_row, s_row, q_col, s_col, s_block};
+  CUtensorMap tm;
+  const int st = encode_bf16_in(&tm, x, static_cast<uint64_t>(cols), static_cast<uint64_t>(rows));
+  if (st != FP8BW_OK) return st;
+  const int tiles = a.tiles_r * a.tiles_c;
+  const int grid = tiles < 2 * sm_count ? tiles : 2 * sm_count;
+  using Kernel = void (*)(CUtensorMap, QuantArgs);
+  static const Kernel kernels[4] = {quant_tile_kernel<kModeRow>, quant_tile_kernel<kModeCol>,
+                                    quant_tile_kernel<kModeRowCol>, quant_tile_kernel<kModeBlock>};
+  static std::once_flag once;
+  static int prep = FP8BW_OK;
+  std::call_once(once, [&]() {
+    for (Kernel k : kernels)
+      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               QuantSmem::kAlloc) != cudaSuccess)
+        prep = FP8BW_ERR_LAUNCH;
+  });
+  if (prep != FP8BW_OK) return prep;
+  const Kernel kernel = kernels[mode >= 0 && mode < 4 ? mode : kModeBlock];
+  kernel<<<grid, kQThreads, QuantSmem::kAlloc, stream>>>(tm, a);
+  return cudaGetLastError() == cudaSuccess ? FP8BW_OK : FP8BW_ERR_LAUNCH;
 }
 
 }  // namespace fp8bw
