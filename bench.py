@@ -81,6 +81,31 @@ def step_gemm_flops():
     return LAYERS * 3 * sum(2 * TOKENS * n * k for _, k, n in kinds())
 
 
+def dist_env():
+    """(world size, rank, local rank) as set by torchrun (1, 0, 0 otherwise)."""
+    return (int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(value, world, device):
+    """The largest `value` over all ranks (an all-reduce MAX); the step time
+    of a multi-GPU run is the slowest rank's."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(world, work_per_rank, seconds):
+    """Whole-job throughput: every rank processes `work_per_rank` units in
+    the (max-over-ranks) time `seconds`."""
+    return world * work_per_rank / seconds
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -147,8 +172,8 @@ class OracleSample:
 
 
 def run_reference(args):
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
+    _, rank, _ = dist_env()
+    if rank != 0:          # the CPU oracle runs once, on rank 0
         return 0
     sample = OracleSample(tokens=64)
     for _ in range(args.warmup):
@@ -313,9 +338,7 @@ def run_gpu(args):
     import torch
     import torch.distributed as dist
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
@@ -372,11 +395,7 @@ def run_gpu(args):
     barrier()
     clk = clocks.stop()
     o.fp8bw_check_device_error(stream)
-    ms = t_start.elapsed_time(t_end) / args.steps
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(t_start.elapsed_time(t_end) / args.steps, world, dev)
 
     # per-kernel durations inside the timed region
     per_kind = {}
@@ -430,12 +449,9 @@ def run_gpu(args):
         torch.cuda.synchronize()
         barrier()
         o.fp8bw_check_device_error(stream)
-        e2e_ms = e_s.elapsed_time(e_e) / args.steps
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": world * flops / (e2e_ms * 1e-3) / 1e12,
+        e2e_ms = max_over_ranks(e_s.elapsed_time(e_e) / args.steps, world,
+                                dev)
+        e2e = {"value": weak_scaling_value(world, flops, e2e_ms * 1e-3) / 1e12,
                "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
@@ -490,7 +506,7 @@ def run_gpu(args):
                "cores": sample.threads, "kind": "oracle",
                "sample": sample.describe(), "seconds": dt}
 
-    value = world * flops / (ms * 1e-3) / 1e12
+    value = weak_scaling_value(world, flops, ms * 1e-3) / 1e12
     line = {
         "metric": METRIC,
         "value": value,
