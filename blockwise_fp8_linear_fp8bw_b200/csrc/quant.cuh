@@ -13,10 +13,12 @@
 // Thread t owns an 8x8 sub-block of the tile: rows 8*(t/16) .. +7, columns
 // 8*(t%16) .. +7, read from shared memory as eight 16-byte vectors. From the
 // registers it derives
-//   * row groups (1x128): the 16 threads of a half-warp share a row, so the
-//     amax is a 4-step xor shuffle; codes leave as 8-byte stores (a half-warp
-//     writes one 128-byte row segment), scales through shared memory as one
-//     512-byte run;
+//   * row groups (1x128): the 16 threads of a half-warp share 8 rows; the
+//     amax is a packed-bf16 max and a 4-step xor shuffle, each row's two
+//     divisions are done once (by one lane of the half-warp) and the qscale
+//     broadcast; codes leave as 8-byte stores (a half-warp writes one
+//     128-byte row segment), scales through shared memory as one 512-byte
+//     run;
 //   * column groups (128x1): per-thread max over its 8 rows, a shuffle with
 //     the other half-warp, then an 8-warp reduction through shared memory; the
 //     transposed codes (8 tokens of one column = 8 bytes per thread) go to a
@@ -92,11 +94,32 @@ __device__ __forceinline__ void group_scale(float amax, float& qscale,
   }
 }
 
+// |x| of two packed bf16 values (clears both sign bits; exact).
+__device__ __forceinline__ uint32_t abs_bf16x2(uint32_t w) { return w & 0x7FFF7FFFu; }
+
+// Element-wise max of two packed non-negative bf16 pairs (exact).
+__device__ __forceinline__ uint32_t max_bf16x2(uint32_t a, uint32_t b) {
+  __nv_bfloat162 r = __hmax2(*reinterpret_cast<__nv_bfloat162*>(&a),
+                             *reinterpret_cast<__nv_bfloat162*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// The larger of the two bf16 halves, as fp32 (exact).
+__device__ __forceinline__ float max_halves(uint32_t w) {
+  return fmaxf(bf16_lo(w), bf16_hi(w));
+}
+
 // Two fp32 values -> two E4M3 codes (round to nearest even, satfinite);
 // `a` lands in the low byte.
 __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
   return static_cast<uint32_t>(
       __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
+}
+
+// x * qscale for the two bf16 values of a packed pair, one IEEE fp32
+// multiply each (round to nearest even), as one f32x2 instruction.
+__device__ __forceinline__ void scale_pair(uint32_t w, float qs, float& t0, float& t1) {
+  fmul2(t0, t1, bf16_lo(w), bf16_hi(w), qs, qs);
 }
 
 // Encode 8 values (already multiplied by qscale) into 8 bytes.
@@ -201,14 +224,14 @@ __global__ void __launch_bounds__(kQThreads, 2)
 
     if constexpr (MODE == kModeBlock) {
       // ---- one amax for the whole 128x128 block -----------------------------
-      float m = 0.0f;
+      uint32_t m2 = 0u;
 #pragma unroll
       for (int p = 0; p < 8; ++p)
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          m = fmaxf(m, fmaxf(fabsf(bf16_lo(v[p][j])), fabsf(bf16_hi(v[p][j]))));
+        for (int j = 0; j < 4; ++j) m2 = max_bf16x2(m2, abs_bf16x2(v[p][j]));
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+      for (int o = 16; o > 0; o >>= 1) m2 = max_bf16x2(m2, __shfl_xor_sync(0xFFFFFFFFu, m2, o));
+      const float m = max_halves(m2);
       if (lane == 0) blk[warp] = m;
       __syncthreads();
       float amax = blk[0];
@@ -222,10 +245,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
         for (int p = 0; p < 8; ++p) {
           float tv[8];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            tv[2 * j] = __fmul_rn(bf16_lo(v[p][j]), qs);
-            tv[2 * j + 1] = __fmul_rn(bf16_hi(v[p][j]), qs);
-          }
+          for (int j = 0; j < 4; ++j) scale_pair(v[p][j], qs, tv[2 * j], tv[2 * j + 1]);
           *reinterpret_cast<uint2*>(a.q_row + (r0 + p) * cols + c0) = pack8(tv);
         }
       }
@@ -234,34 +254,41 @@ __global__ void __launch_bounds__(kQThreads, 2)
         for (int j = 0; j < 8; ++j) {
           float tv[8];
 #pragma unroll
-          for (int p = 0; p < 8; ++p) {
-            const float x = (j & 1) ? bf16_hi(v[p][j >> 1]) : bf16_lo(v[p][j >> 1]);
-            tv[p] = __fmul_rn(x, qs);
+          for (int p = 0; p < 8; p += 2) {
+            const float x0 = (j & 1) ? bf16_hi(v[p][j >> 1]) : bf16_lo(v[p][j >> 1]);
+            const float x1 = (j & 1) ? bf16_hi(v[p + 1][j >> 1]) : bf16_lo(v[p + 1][j >> 1]);
+            fmul2(tv[p], tv[p + 1], x0, x1, qs, qs);
           }
           *reinterpret_cast<uint2*>(T + t_unit_offset(cg * 8 + j, rb)) = pack8(tv);
         }
       }
     } else {
       if constexpr (MODE == kModeRow || MODE == kModeRowCol) {
-        // ---- row groups: 16 lanes of a half-warp share each row ------------
+        // ---- row groups: the 16 lanes of a half-warp share rows 8rb..8rb+7.
+        // amax by packed bf16 max + xor shuffles (every lane gets all 8);
+        // lane (cg & 7) then computes the two divisions of row (cg & 7) and
+        // the qscales are broadcast back by shuffle.
+        float my_amax = 0.0f;
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
-          float m = 0.0f;
+          uint32_t m2 = max_bf16x2(max_bf16x2(abs_bf16x2(v[p][0]), abs_bf16x2(v[p][1])),
+                                   max_bf16x2(abs_bf16x2(v[p][2]), abs_bf16x2(v[p][3])));
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            m = fmaxf(m, fmaxf(fabsf(bf16_lo(v[p][j])), fabsf(bf16_hi(v[p][j]))));
+          for (int o = 8; o > 0; o >>= 1)
+            m2 = max_bf16x2(m2, __shfl_xor_sync(0xFFFFFFFFu, m2, o));
+          const float am = max_halves(m2);
+          if ((cg & 7) == p) my_amax = am;
+        }
+        float my_qs, my_s;
+        group_scale(my_amax, my_qs, my_s);
+        if (cg < 8) srow_s[rb * 8 + cg] = my_s;
 #pragma unroll
-          for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-          float qs, s;
-          group_scale(m, qs, s);
-          if (cg == 0) srow_s[rb * 8 + p] = s;
+        for (int p = 0; p < 8; ++p) {
+          const float qs = __shfl_sync(0xFFFFFFFFu, my_qs, (lane & 16) | p);
           if (cvalid && rvalid) {
             float tv[8];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              tv[2 * j] = __fmul_rn(bf16_lo(v[p][j]), qs);
-              tv[2 * j + 1] = __fmul_rn(bf16_hi(v[p][j]), qs);
-            }
+            for (int j = 0; j < 4; ++j) scale_pair(v[p][j], qs, tv[2 * j], tv[2 * j + 1]);
             *reinterpret_cast<uint2*>(a.q_row + (r0 + p) * cols + c0) = pack8(tv);
           }
         }
@@ -272,17 +299,13 @@ __global__ void __launch_bounds__(kQThreads, 2)
         float cm[8];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          float lo = 0.0f, hi = 0.0f;
+          uint32_t m2 = abs_bf16x2(v[0][j]);
 #pragma unroll
-          for (int p = 0; p < 8; ++p) {
-            lo = fmaxf(lo, fabsf(bf16_lo(v[p][j])));
-            hi = fmaxf(hi, fabsf(bf16_hi(v[p][j])));
-          }
-          cm[2 * j] = lo;
-          cm[2 * j + 1] = hi;
+          for (int p = 1; p < 8; ++p) m2 = max_bf16x2(m2, abs_bf16x2(v[p][j]));
+          m2 = max_bf16x2(m2, __shfl_xor_sync(0xFFFFFFFFu, m2, 16));
+          cm[2 * j] = bf16_lo(m2);
+          cm[2 * j + 1] = bf16_hi(m2);
         }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) cm[j] = fmaxf(cm[j], __shfl_xor_sync(0xFFFFFFFFu, cm[j], 16));
         if (lane < 16) {
           float4* dst = reinterpret_cast<float4*>(&red[warp][cg * 8]);
           dst[0] = make_float4(cm[0], cm[1], cm[2], cm[3]);
@@ -307,9 +330,10 @@ __global__ void __launch_bounds__(kQThreads, 2)
         for (int j = 0; j < 8; ++j) {
           float tv[8];
 #pragma unroll
-          for (int p = 0; p < 8; ++p) {
-            const float x = (j & 1) ? bf16_hi(v[p][j >> 1]) : bf16_lo(v[p][j >> 1]);
-            tv[p] = __fmul_rn(x, qv[j]);
+          for (int p = 0; p < 8; p += 2) {
+            const float x0 = (j & 1) ? bf16_hi(v[p][j >> 1]) : bf16_lo(v[p][j >> 1]);
+            const float x1 = (j & 1) ? bf16_hi(v[p + 1][j >> 1]) : bf16_lo(v[p + 1][j >> 1]);
+            fmul2(tv[p], tv[p + 1], x0, x1, qv[j], qv[j]);
           }
           *reinterpret_cast<uint2*>(T + t_unit_offset(cg * 8 + j, rb)) = pack8(tv);
         }
