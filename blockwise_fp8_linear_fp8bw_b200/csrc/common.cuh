@@ -74,6 +74,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but a thread whose phase is not complete yet is suspended
+// (not spinning on issue slots) until it completes or `suspend_ns` elapse.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Suspension slice of a bounded wait (the abort flag and the time limit are
+// checked between slices).
+constexpr uint32_t kWaitSliceNs = 1000000u;
+
 // Wait for the phase with the given parity to complete. Gives up (returns
 // false) when *abort becomes non-zero or after kWaitLimitNs; on a timeout it
 // records `err_bit` in the device error word and raises *abort so that the
@@ -82,16 +101,14 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           volatile uint32_t* abort,
                                           uint32_t err_bit) {
   if (mbar_try_wait(bar, parity)) return true;
-  uint64_t t0 = globaltimer_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 15u) == 0) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        atomicOr(&g_device_error, err_bit);
-        *abort = 1u;
-        return false;
-      }
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, kWaitSliceNs)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      atomicOr(&g_device_error, err_bit);
+      *abort = 1u;
+      return false;
     }
   }
 }
@@ -188,6 +205,28 @@ __device__ __forceinline__ void fmul2(float& p0, float& p1, float x0, float x1,
       "mov.b64 {%0, %1}, p;\n\t}"
       : "=f"(p0), "=f"(p1)
       : "f"(x0), "f"(x1), "f"(y0), "f"(y1));
+}
+
+// The same packed operations on 64-bit register pairs (lo = first element),
+// for values that stay packed across iterations (accumulators, scale pairs).
+__device__ __forceinline__ uint64_t pack2(uint32_t lo, uint32_t hi) {
+  uint64_t v;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "r"(lo), "r"(hi));
+  return v;
+}
+
+__device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ void ffma2_64(uint64_t& a, uint64_t x, uint64_t s) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(a) : "l"(x), "l"(s));
+}
+
+__device__ __forceinline__ uint64_t fmul2_64(uint64_t x, uint64_t y) {
+  uint64_t p;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(p) : "l"(x), "l"(y));
+  return p;
 }
 
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {

@@ -358,13 +358,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     bool ok = true, store_pending = false;
     for (int tile = cluster_id; ok && tile < num_tiles; tile += num_clusters) {
       const int tm = tile / g.tiles_n, tn = tile % g.tiles_n;
-      float acc[kHalf];
+      uint64_t acc2[kHalf / 2];   // fp32 accumulator pairs (columns 2i, 2i+1)
 #pragma unroll
-      for (int j = 0; j < kHalf; ++j) acc[j] = 0.0f;
+      for (int j = 0; j < kHalf / 2; ++j) acc2[j] = 0ull;
 
       for (int c = 0; c < C; ++c, ++tc, ++sit) {
-        const int tb = tc % kBufs;
-        const uint32_t tu = tc / kBufs;
+        const int tb = tc & 1;
+        const uint32_t tu = tc >> 1;
         const int ss = sit % kScaleStages;
         const uint32_t su = sit / kScaleStages;
         if (!mbar_wait(tfull_bar(tb), tu & 1u, abort_flag, kErrTimeoutEpi) ||
@@ -375,9 +375,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const float* slot = reinterpret_cast<const float*>(smem + L::kScaleOff + ss * L::kScaleSlot);
         const float sa_v = slot[row];
-        const float* sbv = slot + BM;
-        float blk_scale = 0.0f;
-        if constexpr (!VEC_B) blk_scale = sa_v * sbv[BN > 128 ? h : 0];
+        const float* sbv = slot + BM;                 // B scales of this chunk
+        const uint32_t sa_bits = __float_as_uint(sa_v);
+        const uint64_t sa2 = pack2(sa_bits, sa_bits);
+        uint64_t blk2 = 0ull;
+        if constexpr (!VEC_B) {
+          const uint32_t b = __float_as_uint(sa_v * sbv[BN > 128 ? h : 0]);
+          blk2 = pack2(b, b);
+        }
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                static_cast<uint32_t>(tb * BN + h * kHalf);
 #pragma unroll
@@ -387,12 +392,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tmem_ld32(taddr + part * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
           tmem_wait_ld();
           if (part == kHalf / 64 - 1) {
+            // Every TMEM read of this chunk has landed: hand the buffer back to
+            // the MMA warp before doing the arithmetic.
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8u * tb);
           }
-          float* a = acc + part * 64;
+          uint64_t* a = acc2 + part * 32;
           if constexpr (VEC_B) {
+            // (measured: with vector scales the 32-bit form below schedules
+            // better than the packed accumulators, which spill here)
+            float* af = reinterpret_cast<float*>(a);
             const float* sbp = sbv + h * kHalf + part * 64;
 #pragma unroll
             for (int j = 0; j < 64; j += 4) {
@@ -400,20 +410,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               float w0, w1, w2, w3;
               fmul2(w0, w1, sa_v, sa_v, b4.x, b4.y);
               fmul2(w2, w3, sa_v, sa_v, b4.z, b4.w);
-              ffma2(a[j], a[j + 1], __uint_as_float(r[j]), __uint_as_float(r[j + 1]), w0, w1);
-              ffma2(a[j + 2], a[j + 3], __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]), w2, w3);
+              ffma2(af[j], af[j + 1], __uint_as_float(r[j]), __uint_as_float(r[j + 1]), w0, w1);
+              ffma2(af[j + 2], af[j + 3], __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]), w2,
+                    w3);
             }
           } else {
 #pragma unroll
-            for (int j = 0; j < 64; j += 2)
-              ffma2(a[j], a[j + 1], __uint_as_float(r[j]), __uint_as_float(r[j + 1]),
-                    blk_scale, blk_scale);
+            for (int j = 0; j < 32; ++j) ffma2_64(a[j], pack2(r[2 * j], r[2 * j + 1]), blk2);
           }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(sempty_bar(ss));
       }
       if (!ok) break;
+
+      float acc[kHalf];
+#pragma unroll
+      for (int j = 0; j < kHalf / 2; ++j) unpack2(acc2[j], acc[2 * j], acc[2 * j + 1]);
 
       const int y0 = tm * (2 * BM) + static_cast<int>(rank) * BM + q * 32;
       const int x0 = tn * BN + h * kHalf;
