@@ -52,6 +52,37 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
                   "bf16_tflops_sustained": 1400.0}
 FP8_OVER_BF16 = 2.0   # nominal dense FP8 / BF16 tensor throughput (4.5 / 2.25)
 
+# DRAM bytes (read + write) per launch of each kernel, averaged over the 672
+# launches of one step, from one ncu capture (gpu__time_duration.sum,
+# dram__bytes_read.sum, dram__bytes_write.sum; profiles/
+# launches_stack28_m16384.md). Valid only for the kernel sources they were
+# taken on: KERNEL_FINGERPRINT is a hash of csrc/*.cu[h] at that time, and the
+# numbers are reported as null once the sources differ.
+NCU_TRAFFIC_PER_LAUNCH = {
+    "gemm_block_scaled": 183473285,
+    "gemm_vector_scaled": 254376978,
+    "quant_rowcol": 217269387,
+    "quant_weight_block": 25395412,
+}
+KERNEL_FINGERPRINT = "3108ff621dd535ff"
+
+
+def kernel_fingerprint():
+    import hashlib
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "blockwise_fp8_linear_fp8bw_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        if f.endswith((".cu", ".cuh")):
+            with open(os.path.join(d, f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel):
+    if kernel_fingerprint() != KERNEL_FINGERPRINT:
+        return None
+    return NCU_TRAFFIC_PER_LAUNCH.get(kernel)
+
 
 def parse_args():
     p = argparse.ArgumentParser()
@@ -470,6 +501,8 @@ def run_gpu(args):
             ach = d["units"] / (d["ms"] * 1e-3) / 1e12
             breakdown[kk] = {"achieved": ach, "unit": "TFLOP/s",
                              "frac_of_fp8_peak": ach / fp8_sustained,
+                             "flop_per_launch": d["units"] / d["launches"],
+                             "dram_bytes_per_launch_ncu": ncu_traffic(kk),
                              "share": d["ms"] / (ms * args.steps),
                              "launches_per_step": d["launches"] // args.steps,
                              "avg_launch_ms": avg_ms}
@@ -477,6 +510,8 @@ def run_gpu(args):
             ach = d["units"] / (d["ms"] * 1e-3) / 1e9
             breakdown[kk] = {"achieved": ach, "unit": "GB/s",
                              "frac_of_hbm": ach / peaks["hbm_gbs"],
+                             "bytes_per_launch": d["units"] / d["launches"],
+                             "dram_bytes_per_launch_ncu": ncu_traffic(kk),
                              "share": d["ms"] / (ms * args.steps),
                              "launches_per_step": d["launches"] // args.steps,
                              "avg_launch_ms": avg_ms}
@@ -486,14 +521,14 @@ def run_gpu(args):
         ach = dd["units"] / (dd["ms"] * 1e-3) / 1e12
         roofline = {"kernel": dk, "bound": "tensor", "achieved": ach,
                     "peak": fp8_sustained, "unit": "TFLOP/s",
-                    "frac": ach / fp8_sustained, "traffic": None,
+                    "frac": ach / fp8_sustained, "traffic": ncu_traffic(dk),
                     "peak_note": "%s sustained bf16 x %.0f (nominal FP8/BF16)"
                     % (peaks["source"], FP8_OVER_BF16)}
     else:
         ach = dd["units"] / (dd["ms"] * 1e-3) / 1e9
         roofline = {"kernel": dk, "bound": "hbm", "achieved": ach,
                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": ach / peaks["hbm_gbs"], "traffic": None,
+                    "frac": ach / peaks["hbm_gbs"], "traffic": ncu_traffic(dk),
                     "peak_note": "%s copy bandwidth" % peaks["source"]}
 
     cpu = None
