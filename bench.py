@@ -92,6 +92,8 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-next-rows", action="store_true",
+                   help="skip the timing of the rows beyond the step")
     p.add_argument("--layers", type=int, default=28,
                    help="layers per step (profiling runs use fewer)")
     p.add_argument("--linears", default="qkv,o,gate_up,down",
@@ -308,6 +310,43 @@ class LinearBuffers:
         ]
 
 
+def time_next_rows(o, bufs, stream, warmup, rounds):
+    """Rows beyond the step, timed after it on the same buffers (not part of
+    `value`): wgrad with an fp32 dW added into an fp32 main-grad buffer, the
+    four linears of a layer in turn (their operands together exceed L2)."""
+    import torch
+    dev = bufs[0].qx_t.device
+    grads = [torch.zeros((b.n, b.k), dtype=torch.float32, device=dev)
+             for b in bufs]
+    calls = [(2 * TOKENS * b.n * b.k,
+              (lambda b=b, g=g: o.fp8bw_gemm_wgrad_f32(
+                  b.qdy_t, b.sdy_t, b.qx_t, b.sx_t, g, True, stream)))
+             for b, g in zip(bufs, grads)]
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            for _, fn in calls:
+                fn()
+    torch.cuda.synchronize()
+    ev = [[(torch.cuda.Event(enable_timing=True),
+            torch.cuda.Event(enable_timing=True)) for _ in calls]
+          for _ in range(rounds)]
+    with torch.cuda.stream(stream):
+        for r in range(rounds):
+            for (_, fn), (e0, e1) in zip(calls, ev[r]):
+                e0.record(stream)
+                fn()
+                e1.record(stream)
+    torch.cuda.synchronize()
+    o.fp8bw_check_device_error(stream)
+    ms = sum(e0.elapsed_time(e1) for r in ev for e0, e1 in r)
+    flop = rounds * sum(f for f, _ in calls)
+    return {"wgrad_f32_accumulate": {
+        "achieved": flop / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "launches": rounds * len(calls), "avg_launch_ms": ms / (rounds * len(calls)),
+        "what": "dW (fp32) += dY^T X for the QKV, O, gate/up and down "
+                "linears at M=%d, in turn; timed after the step" % TOKENS}}
+
+
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,"
               "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
@@ -437,6 +476,10 @@ def run_gpu(args):
             d["units"] += units
             d["launches"] += 1
 
+    next_rows = None
+    if not args.no_next_rows:
+        next_rows = time_next_rows(o, bufs, stream, args.warmup, 5)
+
     # ---------------------------------------------------------- end to end
     e2e = None
     if not args.no_e2e:
@@ -541,6 +584,9 @@ def run_gpu(args):
                "cores": sample.threads, "kind": "oracle",
                "sample": sample.describe(), "seconds": dt}
 
+    if next_rows is not None:
+        for d in next_rows.values():
+            d["frac_of_fp8_peak"] = d["achieved"] / fp8_sustained
     value = weak_scaling_value(world, flops, ms * 1e-3) / 1e12
     line = {
         "metric": METRIC,
@@ -566,6 +612,7 @@ def run_gpu(args):
         "gpu_launches": len(step_ops) * args.steps,
         "roofline": roofline,
         "breakdown": breakdown,
+        "next_rows": next_rows,
         "clocks": clk,
         "e2e": e2e,
         "cpu_baseline": cpu,

@@ -143,6 +143,22 @@ int encode_bf16_out(CUtensorMap* map, void* base, uint64_t cols, uint64_t rows) 
   return r == CUDA_SUCCESS ? FP8BW_OK : FP8BW_ERR_CUDA;
 }
 
+// 2-D fp32 output tensor [rows, cols] written (or added to) in 16 x 32 boxes
+// (64-byte rows, 64-byte swizzle); out-of-range parts of a box are skipped.
+int encode_f32_out(CUtensorMap* map, void* base, uint64_t cols, uint64_t rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  int st = get_encode(&enc);
+  if (st != FP8BW_OK) return st;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 4};
+  cuuint32_t box[2] = {16u, 32u};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FP8BW_OK : FP8BW_ERR_CUDA;
+}
+
 // --------------------------------------------------------------- GEMM launch
 struct GemmProblem {
   const uint8_t* a;  // [mo][kc]
@@ -153,14 +169,15 @@ struct GemmProblem {
   const float* sa;
   const float* sb;
   int64_t sbj, sbc;
-  uint16_t* out;
+  void* out;         // [mo][no]: bf16 (kOutBf16) or fp32
+  int out_mode;      // gemm::kOutBf16 / kOutF32 / kOutF32Add
 };
 
 // CTA-pair kernel: 256 x 256 output tiles on clusters of two CTAs.
-template <int BN, bool VEC_B, bool B_MN>
+template <int BN, bool VEC_B, bool B_MN, int OUT = gemm::kOutBf16>
 int launch_gemm_pair(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t stream) {
   using L = gemm::PairLayout<BN, VEC_B>;
-  auto kernel = gemm::blockwise_gemm_pair_kernel<BN, VEC_B, B_MN>;
+  auto kernel = gemm::blockwise_gemm_pair_kernel<BN, VEC_B, B_MN, OUT>;
   static std::once_flag once;
   static int prep_status = FP8BW_OK;
   static int max_clusters = 0;
@@ -206,7 +223,11 @@ int launch_gemm_pair(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t s
     st = encode_u8_2d(&tm_b, p.b, static_cast<uint64_t>(p.kc), static_cast<uint64_t>(p.no),
                       BN / 2);
   if (st != FP8BW_OK) return st;
-  st = encode_bf16_out(&tm_out, p.out, static_cast<uint64_t>(p.no), static_cast<uint64_t>(p.mo));
+  if (OUT == gemm::kOutBf16)
+    st = encode_bf16_out(&tm_out, p.out, static_cast<uint64_t>(p.no),
+                         static_cast<uint64_t>(p.mo));
+  else
+    st = encode_f32_out(&tm_out, p.out, static_cast<uint64_t>(p.no), static_cast<uint64_t>(p.mo));
   if (st != FP8BW_OK) return st;
 
   gemm::Args g;
@@ -234,11 +255,20 @@ int run_gemm(const GemmProblem& p, cudaStream_t stream) {
   if (st != FP8BW_OK) return st;
   if (p.mo == 0 || p.no == 0) return FP8BW_OK;
   if (p.kc == 0) {
-    return cudaMemsetAsync(p.out, 0, static_cast<size_t>(p.mo * p.no * 2), stream) == cudaSuccess
+    // An empty contraction: the product is zero (adding it changes nothing).
+    if (p.out_mode == gemm::kOutF32Add) return FP8BW_OK;
+    const size_t esize = p.out_mode == gemm::kOutBf16 ? 2 : 4;
+    return cudaMemsetAsync(p.out, 0, static_cast<size_t>(p.mo * p.no) * esize, stream) ==
+                   cudaSuccess
                ? FP8BW_OK
                : FP8BW_ERR_CUDA;
   }
   if (cdiv(p.mo, 256) * cdiv(p.no, 256) > (int64_t(1) << 30)) return FP8BW_ERR_SHAPE;
+  if (p.vec_b && p.out_mode == gemm::kOutF32)
+    return launch_gemm_pair<GEMM_BN_VEC, true, false, gemm::kOutF32>(p, dev, stream);
+  if (p.vec_b && p.out_mode == gemm::kOutF32Add)
+    return launch_gemm_pair<GEMM_BN_VEC, true, false, gemm::kOutF32Add>(p, dev, stream);
+  if (p.out_mode != gemm::kOutBf16) return FP8BW_ERR_LAUNCH;
   if (p.vec_b) return launch_gemm_pair<GEMM_BN_VEC, true, false>(p, dev, stream);
   if (p.b_mn) return launch_gemm_pair<256, false, true>(p, dev, stream);
   return launch_gemm_pair<GEMM_BN_BLOCK, false, false>(p, dev, stream);
@@ -251,7 +281,7 @@ using namespace fp8bw;
 
 extern "C" {
 
-int fp8bw_version(void) { return 100; }
+int fp8bw_version(void) { return 101; }
 
 const char* fp8bw_status_string(int status) {
   switch (status) {
@@ -384,9 +414,13 @@ int fp8bw_gemm_dgrad(const uint8_t* qdy, const float* sdy, const uint8_t* qw,
   return run_gemm(p, static_cast<cudaStream_t>(stream));
 }
 
-int fp8bw_gemm_wgrad(const uint8_t* qdy_t, const float* sdy_t, const uint8_t* qx_t,
-                     const float* sx_t, int64_t m, int64_t n, int64_t k, uint16_t* dw,
-                     void* stream) {
+}  // extern "C"
+
+namespace {
+
+int wgrad_common(const uint8_t* qdy_t, const float* sdy_t, const uint8_t* qx_t,
+                 const float* sx_t, int64_t m, int64_t n, int64_t k, void* dw, int out_mode,
+                 void* stream) {
   if (!dim_ok(m) || !dim_ok(n) || !dim_ok(k)) return FP8BW_ERR_SHAPE;
   if (missing(qdy_t, n * m) || missing(sdy_t, cdiv(m, 128) * n) || missing(qx_t, k * m) ||
       missing(sx_t, cdiv(m, 128) * k) || missing(dw, n * k))
@@ -394,7 +428,8 @@ int fp8bw_gemm_wgrad(const uint8_t* qdy_t, const float* sdy_t, const uint8_t* qx
   if (!aligned16(qdy_t) || !aligned16(sdy_t) || !aligned16(qx_t) || !aligned16(sx_t) ||
       !aligned16(dw))
     return FP8BW_ERR_ALIGN;
-  const Range rd = range_of(dw, n * k * 2);
+  const int64_t esize = out_mode == gemm::kOutBf16 ? 2 : 4;
+  const Range rd = range_of(dw, n * k * esize);
   if (overlap(rd, range_of(qdy_t, n * m)) || overlap(rd, range_of(sdy_t, cdiv(m, 128) * n * 4)) ||
       overlap(rd, range_of(qx_t, k * m)) || overlap(rd, range_of(sx_t, cdiv(m, 128) * k * 4)))
     return FP8BW_ERR_ALIAS;
@@ -411,7 +446,25 @@ int fp8bw_gemm_wgrad(const uint8_t* qdy_t, const float* sdy_t, const uint8_t* qx
   p.sbj = 0;
   p.sbc = 0;
   p.out = dw;
+  p.out_mode = out_mode;
   return run_gemm(p, static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+int fp8bw_gemm_wgrad(const uint8_t* qdy_t, const float* sdy_t, const uint8_t* qx_t,
+                     const float* sx_t, int64_t m, int64_t n, int64_t k, uint16_t* dw,
+                     void* stream) {
+  return wgrad_common(qdy_t, sdy_t, qx_t, sx_t, m, n, k, dw, gemm::kOutBf16, stream);
+}
+
+int fp8bw_gemm_wgrad_f32(const uint8_t* qdy_t, const float* sdy_t, const uint8_t* qx_t,
+                         const float* sx_t, int64_t m, int64_t n, int64_t k, float* dw,
+                         int accumulate, void* stream) {
+  return wgrad_common(qdy_t, sdy_t, qx_t, sx_t, m, n, k, dw,
+                      accumulate ? gemm::kOutF32Add : gemm::kOutF32, stream);
 }
 
 int fp8bw_check_device_error(void* stream) {

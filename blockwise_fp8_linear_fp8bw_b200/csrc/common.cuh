@@ -160,6 +160,17 @@ __device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src,
       : "memory");
 }
 
+// Element-wise add of a shared-memory box into global memory (the add happens
+// at L2; an f32 tensor map adds in fp32). Same coordinate rules as the store.
+__device__ __forceinline__ void tma_reduce_add_2d(const void* tmap, uint32_t src,
+                                                  int32_t x, int32_t y) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group "
+      "[%0, {%1, %2}], [%3];" ::"l"(reinterpret_cast<uint64_t>(tmap)),
+      "r"(x), "r"(y), "r"(src)
+      : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit_group() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }

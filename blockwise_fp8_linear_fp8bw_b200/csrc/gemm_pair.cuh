@@ -40,8 +40,11 @@
 //               loads the partial sums with tcgen05.ld, hands the buffer back,
 //               and adds them, times the two scales, into fp32 accumulators
 //               held in registers (BN/2 per thread; packed f32x2 arithmetic);
-//               after the last chunk it converts to bf16, stages 32x32 boxes
-//               in shared memory and writes them with TMA stores.
+//               after the last chunk it stages the tile in shared memory, box
+//               by box, and writes it with TMA: bf16 32x32 boxes (the GEMM's
+//               output), or fp32 16-column x 32-row boxes, either stored or
+//               added element-wise into the fp32 tensor already in memory
+//               (a weight-gradient accumulator).
 // With BN = 256 the producer warps give registers to the promotion warps
 // (setmaxnreg 56 / 224: 4*32*56 + 8*32*224 = 384 * 168, the launch budget).
 // Every mbarrier wait is bounded (about 2 s, common.cuh); on expiry the CTA
@@ -73,6 +76,11 @@ static_assert(4 * 32 * kProducerRegs + kNumEpiWarps * 32 * kEpilogueRegs ==
                   kThreads * kLaunchRegs,
               "setmaxnreg split must equal the launch register budget");
 
+// Output modes of the epilogue.
+constexpr int kOutBf16 = 0;       // bf16 store
+constexpr int kOutF32 = 1;        // fp32 store
+constexpr int kOutF32Add = 2;     // fp32 add into the existing output (TMA reduce-add)
+
 struct Args {
   int mo, no, kc;             // output rows, output columns, contraction length
   int tiles_m, tiles_n, chunks;
@@ -80,7 +88,7 @@ struct Args {
   const float* sb;            // vector: [chunks][no]; block: sb[jb*sbj + c*sbc]
   int64_t sbj, sbc;
   int nblk;                   // number of 128-wide output column blocks
-  uint16_t* out;              // bf16 [mo][no]
+  void* out;                  // [mo][no], bf16 or fp32 (written through tm_out)
 };
 
 __device__ __forceinline__ void setmaxnreg_dec() {
@@ -120,7 +128,7 @@ struct PairLayout {
   static_assert(kAlloc <= 227 * 1024, "shared memory budget");
 };
 
-template <int BN_, bool VEC_B, bool B_MN>
+template <int BN_, bool VEC_B, bool B_MN, int OUT = kOutBf16>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     blockwise_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
                                const __grid_constant__ CUtensorMap tm_b,
@@ -430,20 +438,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
       const int y0 = tm * (2 * BM) + static_cast<int>(rank) * BM + q * 32;
       const int x0 = tn * BN + h * kHalf;
+      // One 2 KB staging box per warp: 32 rows of 64 bytes (32 bf16 or 16
+      // fp32 columns), 64-byte swizzle (16-byte unit j of row r at j ^ (r/2 % 4)).
+      constexpr int kBoxCols = OUT == kOutBf16 ? 32 : 16;
 #pragma unroll
-      for (int gi = 0; gi < kHalf / 32; ++gi) {
-        if (x0 + gi * 32 >= g.no || y0 >= g.mo) continue;
+      for (int gi = 0; gi < kHalf / kBoxCols; ++gi) {
+        if (x0 + gi * kBoxCols >= g.no || y0 >= g.mo) continue;
         if (store_pending) {
           if (lane == 0) bulk_wait_group_read<0>();
           __syncwarp();
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const float* v = acc + gi * 32 + j * 8;
-          const uint32_t w0 = pack_bf16x2(v[0], v[1]);
-          const uint32_t w1 = pack_bf16x2(v[2], v[3]);
-          const uint32_t w2 = pack_bf16x2(v[4], v[5]);
-          const uint32_t w3 = pack_bf16x2(v[6], v[7]);
+          uint32_t w0, w1, w2, w3;
+          if constexpr (OUT == kOutBf16) {
+            const float* v = acc + gi * 32 + j * 8;
+            w0 = pack_bf16x2(v[0], v[1]);
+            w1 = pack_bf16x2(v[2], v[3]);
+            w2 = pack_bf16x2(v[4], v[5]);
+            w3 = pack_bf16x2(v[6], v[7]);
+          } else {
+            const float* v = acc + gi * 16 + j * 4;
+            w0 = __float_as_uint(v[0]);
+            w1 = __float_as_uint(v[1]);
+            w2 = __float_as_uint(v[2]);
+            w3 = __float_as_uint(v[3]);
+          }
           const uint32_t dst = stage_out + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4);
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(w0),
                        "r"(w1), "r"(w2), "r"(w3)
@@ -452,7 +472,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&tm_out, stage_out, x0 + gi * 32, y0);
+          if constexpr (OUT == kOutF32Add)
+            tma_reduce_add_2d(&tm_out, stage_out, x0 + gi * kBoxCols, y0);
+          else
+            tma_store_2d(&tm_out, stage_out, x0 + gi * kBoxCols, y0);
           bulk_commit_group();
         }
         store_pending = true;

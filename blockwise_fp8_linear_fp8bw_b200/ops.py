@@ -136,6 +136,20 @@ def fp8bw_gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t, dw, stream=None):
            "fp8bw_gemm_wgrad")
 
 
+def fp8bw_gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, dw, accumulate=False,
+                         stream=None):
+    n, m = qdy_t.shape
+    k = qx_t.shape[0]
+    _expect(qx_t, torch.uint8, (k, m), "qx_t")
+    _expect(sdy_t, torch.float32, (_cdiv(m, 128), n), "sdy_t")
+    _expect(sx_t, torch.float32, (_cdiv(m, 128), k), "sx_t")
+    _expect(dw, torch.float32, (n, k), "dw")
+    _check(_lib.fp8bw_gemm_wgrad_f32(_ptr(qdy_t), _ptr(sdy_t), _ptr(qx_t),
+                                     _ptr(sx_t), m, n, k, _ptr(dw),
+                                     1 if accumulate else 0, _stream(stream)),
+           "fp8bw_gemm_wgrad_f32")
+
+
 def fp8bw_check_device_error(stream=None):
     _check(_lib.fp8bw_check_device_error(_stream(stream)),
            "fp8bw_check_device_error")
@@ -199,4 +213,16 @@ def gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t, stream=None):
     dw = torch.empty((qdy_t.shape[0], qx_t.shape[0]), dtype=torch.bfloat16,
                      device=qdy_t.device)
     fp8bw_gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t, dw, stream)
+    return dw
+
+
+def gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, main_grad=None, stream=None):
+    """fp32 dW; with `main_grad` given, dW is added into it in place and it is
+    returned."""
+    if main_grad is not None:
+        fp8bw_gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, main_grad, True, stream)
+        return main_grad
+    dw = torch.empty((qdy_t.shape[0], qx_t.shape[0]), dtype=torch.float32,
+                     device=qdy_t.device)
+    fp8bw_gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, dw, False, stream)
     return dw

@@ -139,6 +139,25 @@ int fp8bw_gemm_wgrad(const uint8_t* qdy_t, const float* sdy_t,
                      const uint8_t* qx_t, const float* sx_t, int64_t m,
                      int64_t n, int64_t k, uint16_t* dw, void* stream);
 
+/* wgrad with an fp32 weight gradient: the same sum as fp8bw_gemm_wgrad, kept
+ * in fp32 (no bf16 rounding), for the fp32 main-grad of mixed-precision
+ * training.
+ *   accumulate == 0 : dW := P           (dw is write-only)
+ *   accumulate != 0 : dW := fp32(dW + P) element-wise, P being the fp32 sum
+ *                     above; dw must hold the previous gradient (e.g. the
+ *                     other micro-batches' sum). The add is done in memory,
+ *                     by the TMA unit, once per element per call.
+ *   dw : fp32 [n, k], caller-owned device memory, 16-byte aligned, must not
+ *        overlap any input. Other arguments and errors as fp8bw_gemm_wgrad;
+ *        m == 0 writes zeros (accumulate == 0) or leaves dw unchanged.
+ * Source: paperlayer.ai summary, Appendix C, "FP8 implementation pipeline"
+ * (gradients are kept in FP32; the weight-gradient GEMM is one of the FP8
+ * GEMMs). */
+int fp8bw_gemm_wgrad_f32(const uint8_t* qdy_t, const float* sdy_t,
+                         const uint8_t* qx_t, const float* sx_t, int64_t m,
+                         int64_t n, int64_t k, float* dw, int accumulate,
+                         void* stream);
+
 /* Synchronises `stream`, then returns FP8BW_ERR_DEVICE_TIMEOUT if any kernel
  * of this library on the current device recorded an expired wait since the
  * last call (and clears the record), else FP8BW_OK (or FP8BW_ERR_CUDA if the

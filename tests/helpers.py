@@ -49,6 +49,29 @@ def assert_gemm_close(got_bits, acc, bound, what=""):
                         got[bad][:5], np.asarray(acc)[bad][:5], tol[bad][:5]))
 
 
+def ulp_f32(v):
+    """Spacing of fp32 at |v|: 2^(max(floor(log2|v|), -126) - 23)."""
+    v = np.abs(np.asarray(v, np.float64))
+    e = np.full(v.shape, -126.0)
+    nz = v > 0
+    e[nz] = np.maximum(np.floor(np.log2(v[nz])), -126.0)
+    return np.exp2(e - 23.0)
+
+
+def assert_gemm_close_f32(got, ref, bound, what=""):
+    """fp32 outputs: |got - ref| <= 1e-3 * sum_k |a_k b_k| + 1 fp32 ulp(ref)."""
+    got = np.asarray(got, np.float64)
+    err = np.abs(got - ref)
+    tol = 1e-3 * np.asarray(bound) + ulp_f32(ref)
+    bad = ~(err <= tol)
+    if bad.any():
+        idx = np.argwhere(bad)[:5]
+        raise AssertionError(
+            "%s: %d of %d elements outside tolerance; first %s: got %s ref %s "
+            "tol %s" % (what, int(bad.sum()), bad.size, idx.tolist(),
+                        got[bad][:5], np.asarray(ref)[bad][:5], tol[bad][:5]))
+
+
 def sample_points(rows, cols, seed=0, per_tile=16, stripes=2, tile=128):
     """At least `per_tile` seeded points in every 128x128 output tile, plus
     `stripes` full rows and full columns."""
@@ -75,5 +98,6 @@ def scale_bits(s):
 
 
 __all__ = ["bf16_np_to_torch", "torch_bf16_to_np", "bf16_bits_to_f64",
-           "ulp_bf16", "gemm_tolerance", "assert_gemm_close",
+           "ulp_bf16", "gemm_tolerance", "assert_gemm_close", "ulp_f32",
+           "assert_gemm_close_f32",
            "sample_points", "scale_bits", "oracle"]

@@ -36,14 +36,14 @@ def lib():
 
 def test_every_declared_symbol_is_exported(lib):
     names = declared_functions()
-    assert len(names) == 9
+    assert len(names) == 10
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(_native.SIGNATURES)
 
 
 def test_status_strings_and_version(lib):
-    assert lib.fp8bw_version() == 100
+    assert lib.fp8bw_version() == 101
     for st in (OK, E_NULL, E_SHAPE, E_ALIGN, E_DEVICE, E_LAUNCH, E_TIMEOUT,
                E_CUDA, E_ALIAS):
         s = lib.fp8bw_status_string(st).decode()
@@ -66,6 +66,8 @@ def test_null_pointers_rejected(lib):
                                 None) == E_NULL
     assert lib.fp8bw_gemm_wgrad(A, B, C, D, 128, 128, 128, None,
                                 None) == E_NULL
+    assert lib.fp8bw_gemm_wgrad_f32(A, B, C, D, 128, 128, 128, None, 1,
+                                    None) == E_NULL
 
 
 @pytest.mark.parametrize("rows,cols", [(-16, 128), (128, -16), (100, 128),
@@ -82,6 +84,8 @@ def test_bad_shapes_rejected(lib, rows, cols):
                                 None) == E_SHAPE
     assert lib.fp8bw_gemm_wgrad(A, B, C, D, cols, 128, rows, E,
                                 None) == E_SHAPE
+    assert lib.fp8bw_gemm_wgrad_f32(A, B, C, D, cols, 128, rows, E, 0,
+                                    None) == E_SHAPE
 
 
 def test_misaligned_pointers_rejected(lib):
@@ -96,6 +100,8 @@ def test_misaligned_pointers_rejected(lib):
                                 None) == E_ALIGN
     assert lib.fp8bw_gemm_wgrad(A, B, C, D + 4, 128, 128, 128, E,
                                 None) == E_ALIGN
+    assert lib.fp8bw_gemm_wgrad_f32(A, B, C, D, 128, 128, 128, E + 8, 1,
+                                    None) == E_ALIGN
 
 
 def test_aliased_outputs_rejected(lib):
@@ -106,6 +112,11 @@ def test_aliased_outputs_rejected(lib):
                                 None) == E_ALIAS
     assert lib.fp8bw_gemm_wgrad(A, B, C, D, 128, 128, 128, C + 256,
                                 None) == E_ALIAS
+    # the fp32 dW is 4 bytes per element: [C - 128*128*4 + 16, C + 16)
+    # reaches into qX^T at C
+    assert lib.fp8bw_gemm_wgrad_f32(A, B, C, D, 128, 128, 128,
+                                    C - 128 * 128 * 4 + 16, 1,
+                                    None) == E_ALIAS
 
 
 @pytest.mark.skipif(
@@ -115,3 +126,5 @@ def test_valid_call_without_device_reports_device_error(lib):
     assert lib.fp8bw_quantize_rowwise(A, 128, 128, B, C, None) == E_DEVICE
     assert lib.fp8bw_gemm_fprop(A, B, C, D, 128, 128, 128, E,
                                 None) == E_DEVICE
+    assert lib.fp8bw_gemm_wgrad_f32(A, B, C, D, 128, 128, 128, E, 1,
+                                    None) == E_DEVICE
