@@ -135,3 +135,20 @@ def test_full_size_mlp_backward():
                 full=False)
     _wgrad_case(16384, 12288, 2048, S.tensor_id("gate_up", "dy"), full=False)
     _ops().fp8bw_check_device_error()
+
+
+@pytest.mark.parametrize("m,n,k", [(272, 400, 528), (16384, 2048, 2048)])
+def test_wgrad_repeatable(m, n, k):
+    """Repeated weight-gradient calls on the same operands give the same
+    bits (no order-dependent accumulation anywhere in the kernel)."""
+    import torch
+    ops = _ops()
+    dy = S.bf16_normal((m, n), 0, 641, **S.DY_DIST)
+    x = S.bf16_normal((m, k), 0, 642, **S.X_DIST)
+    qdy_t, sdy_t = ops.quantize_colwise(bf16_np_to_torch(dy))
+    qx_t, sx_t = ops.quantize_colwise(bf16_np_to_torch(x))
+    first = ops.gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t)
+    for _ in range(3):
+        again = ops.gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t)
+        assert torch.equal(again.view(torch.int16), first.view(torch.int16))
+    ops.fp8bw_check_device_error()
