@@ -184,6 +184,35 @@ void orc_group_scale(float amax, float* qscale, float* s)
     *s = amax / 448.0f;                   /* dequantisation scale */
 }
 
+/* Power-of-two variant (the form the B200 tensor cores apply in hardware,
+ * UE8M0 scale factors; the pages leave the scale form open -- the arxiv-wiki
+ * summary's developer notes only say the grouping and scaling follow the
+ * DeepSeek-V3 approach). s = 2^E with E the smallest integer such that
+ * 448 * 2^E >= amax, clamped to [-127, 127]; qscale = 2^-E. amax == 0 or a
+ * non-finite amax gives qscale = s = 1. The test 448 * 2^E >= amax is exact
+ * in binary64. */
+void orc_group_scale_pow2(float amax, float* qscale, float* s)
+{
+    int e;
+    if (amax == 0.0f || !isfinite(amax)) {
+        *qscale = 1.0f;
+        *s = 1.0f;
+        return;
+    }
+    /* start near log2(amax / 448) and step to the smallest valid E */
+    (void)frexp((double)amax / 448.0, &e);
+    while (ldexp(448.0, e) < (double)amax)
+        ++e;
+    while (ldexp(448.0, e - 1) >= (double)amax)
+        --e;
+    if (e < -127)
+        e = -127;
+    if (e > 127)
+        e = 127;
+    *qscale = (float)ldexp(1.0, -e);      /* exact: a power of two in range */
+    *s = (float)ldexp(1.0, e);            /* 2^-127 is a binary32 subnormal */
+}
+
 /* Encode one element of a group: t = x * qscale in binary32, then E4M3. */
 static uint8_t encode_elem(uint16_t xb, float qscale)
 {
@@ -195,8 +224,10 @@ static int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 /* Row-wise 1x128 activation quantiser: groups run along the columns (the
  * contraction dimension of the GEMM that consumes the codes). */
-int orc_quantize_rowwise(const uint16_t* x, int64_t rows, int64_t cols,
-                         uint8_t* q, float* s)
+typedef void (*scale_fn)(float, float*, float*);
+
+static int quantize_rowwise(const uint16_t* x, int64_t rows, int64_t cols,
+                            uint8_t* q, float* s, scale_fn scale)
 {
     int64_t r, g, c, ngroups;
     if (!x || !q || !s || rows < 0 || cols < 0)
@@ -211,7 +242,7 @@ int orc_quantize_rowwise(const uint16_t* x, int64_t rows, int64_t cols,
                 if (a > amax)
                     amax = a;
             }
-            orc_group_scale(amax, &qscale, &sc);
+            scale(amax, &qscale, &sc);
             for (c = c0; c < c1; ++c)
                 q[r * cols + c] = encode_elem(x[r * cols + c], qscale);
             s[g * rows + r] = sc;
@@ -224,8 +255,8 @@ int orc_quantize_rowwise(const uint16_t* x, int64_t rows, int64_t cols,
  * which is the contraction dimension of the weight-gradient GEMM -- paperlayer.ai
  * summary, Appendix C, "FP8 implementation pipeline"). Codes are written
  * transposed: q_t[col][row]. */
-int orc_quantize_colwise(const uint16_t* x, int64_t rows, int64_t cols,
-                         uint8_t* q_t, float* s_t)
+static int quantize_colwise(const uint16_t* x, int64_t rows, int64_t cols,
+                            uint8_t* q_t, float* s_t, scale_fn scale)
 {
     int64_t r, g, c, ngroups;
     if (!x || !q_t || !s_t || rows < 0 || cols < 0)
@@ -240,7 +271,7 @@ int orc_quantize_colwise(const uint16_t* x, int64_t rows, int64_t cols,
                 if (a > amax)
                     amax = a;
             }
-            orc_group_scale(amax, &qscale, &sc);
+            scale(amax, &qscale, &sc);
             for (r = r0; r < r1; ++r)
                 q_t[c * rows + r] = encode_elem(x[r * cols + c], qscale);
             s_t[g * cols + c] = sc;
@@ -251,8 +282,9 @@ int orc_quantize_colwise(const uint16_t* x, int64_t rows, int64_t cols,
 
 /* Weight quantiser, one scale per 128x128 block (arxiv-wiki summary, Approach
  * item (4)). q_t, when not NULL, receives the same codes transposed. */
-int orc_quantize_weight_block(const uint16_t* w, int64_t n, int64_t k,
-                              uint8_t* q, float* s, uint8_t* q_t)
+static int quantize_weight_block(const uint16_t* w, int64_t n, int64_t k,
+                                 uint8_t* q, float* s, uint8_t* q_t,
+                                 scale_fn scale)
 {
     int64_t nb, kb, i, j, nblk_n, nblk_k;
     if (!w || !q || !s || n < 0 || k < 0)
@@ -270,7 +302,7 @@ int orc_quantize_weight_block(const uint16_t* w, int64_t n, int64_t k,
                     if (a > amax)
                         amax = a;
                 }
-            orc_group_scale(amax, &qscale, &sc);
+            scale(amax, &qscale, &sc);
             for (i = i0; i < i1; ++i)
                 for (j = j0; j < j1; ++j) {
                     uint8_t code = encode_elem(w[i * k + j], qscale);
@@ -282,6 +314,42 @@ int orc_quantize_weight_block(const uint16_t* w, int64_t n, int64_t k,
         }
     }
     return 0;
+}
+
+int orc_quantize_rowwise(const uint16_t* x, int64_t rows, int64_t cols,
+                         uint8_t* q, float* s)
+{
+    return quantize_rowwise(x, rows, cols, q, s, orc_group_scale);
+}
+
+int orc_quantize_colwise(const uint16_t* x, int64_t rows, int64_t cols,
+                         uint8_t* q_t, float* s_t)
+{
+    return quantize_colwise(x, rows, cols, q_t, s_t, orc_group_scale);
+}
+
+int orc_quantize_weight_block(const uint16_t* w, int64_t n, int64_t k,
+                              uint8_t* q, float* s, uint8_t* q_t)
+{
+    return quantize_weight_block(w, n, k, q, s, q_t, orc_group_scale);
+}
+
+int orc_quantize_rowwise_pow2(const uint16_t* x, int64_t rows, int64_t cols,
+                              uint8_t* q, float* s)
+{
+    return quantize_rowwise(x, rows, cols, q, s, orc_group_scale_pow2);
+}
+
+int orc_quantize_colwise_pow2(const uint16_t* x, int64_t rows, int64_t cols,
+                              uint8_t* q_t, float* s_t)
+{
+    return quantize_colwise(x, rows, cols, q_t, s_t, orc_group_scale_pow2);
+}
+
+int orc_quantize_weight_block_pow2(const uint16_t* w, int64_t n, int64_t k,
+                                   uint8_t* q, float* s, uint8_t* q_t)
+{
+    return quantize_weight_block(w, n, k, q, s, q_t, orc_group_scale_pow2);
 }
 
 /* ------------------------------------------------------------------------ */

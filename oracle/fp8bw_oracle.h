@@ -48,6 +48,10 @@ void    orc_e4m3_encode_array(const float* t, int64_t count, uint8_t* out);
 
 /* Group scale pair from an amax (see header comment). */
 void orc_group_scale(float amax, float* qscale, float* s);
+/* Power-of-two variant: s = 2^E, E the smallest integer with 448 * 2^E >=
+ * amax, clamped to [-127, 127]; qscale = 2^-E; amax == 0 or non-finite gives
+ * qscale = s = 1. */
+void orc_group_scale_pow2(float amax, float* qscale, float* s);
 
 /* bf16 helpers (raw bit patterns). */
 float    orc_bf16_to_float(uint16_t b);
@@ -60,6 +64,13 @@ int orc_quantize_colwise(const uint16_t* x, int64_t rows, int64_t cols,
                          uint8_t* q_t, float* s_t);
 int orc_quantize_weight_block(const uint16_t* w, int64_t n, int64_t k,
                               uint8_t* q, float* s, uint8_t* q_t);
+/* The same quantisers with power-of-two scales (orc_group_scale_pow2). */
+int orc_quantize_rowwise_pow2(const uint16_t* x, int64_t rows, int64_t cols,
+                              uint8_t* q, float* s);
+int orc_quantize_colwise_pow2(const uint16_t* x, int64_t rows, int64_t cols,
+                              uint8_t* q_t, float* s_t);
+int orc_quantize_weight_block_pow2(const uint16_t* w, int64_t n, int64_t k,
+                                   uint8_t* q, float* s, uint8_t* q_t);
 
 /* GEMMs, full output.  acc and bound are fp64 [rows_out][cols_out]; bound is
  * sum_k |a_k * b_k| of the dequantised operands (may be NULL). nthreads <= 1

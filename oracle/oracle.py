@@ -37,17 +37,21 @@ def _L():
         lib.orc_e4m3_encode.restype = ctypes.c_uint8
         lib.orc_e4m3_encode_array.argtypes = [P, I64, P]
         lib.orc_e4m3_encode_array.restype = None
-        lib.orc_group_scale.argtypes = [ctypes.c_float, P, P]
-        lib.orc_group_scale.restype = None
+        for name in ("orc_group_scale", "orc_group_scale_pow2"):
+            getattr(lib, name).argtypes = [ctypes.c_float, P, P]
+            getattr(lib, name).restype = None
         lib.orc_bf16_round.argtypes = [ctypes.c_double]
         lib.orc_bf16_round.restype = ctypes.c_uint16
         lib.orc_bf16_to_float.argtypes = [ctypes.c_uint16]
         lib.orc_bf16_to_float.restype = ctypes.c_float
-        for name in ("orc_quantize_rowwise", "orc_quantize_colwise"):
+        for name in ("orc_quantize_rowwise", "orc_quantize_colwise",
+                     "orc_quantize_rowwise_pow2", "orc_quantize_colwise_pow2"):
             getattr(lib, name).argtypes = [P, I64, I64, P, P]
             getattr(lib, name).restype = ctypes.c_int
-        lib.orc_quantize_weight_block.argtypes = [P, I64, I64, P, P, P]
-        lib.orc_quantize_weight_block.restype = ctypes.c_int
+        for name in ("orc_quantize_weight_block",
+                     "orc_quantize_weight_block_pow2"):
+            getattr(lib, name).argtypes = [P, I64, I64, P, P, P]
+            getattr(lib, name).restype = ctypes.c_int
         for name in ("orc_gemm_fprop", "orc_gemm_dgrad", "orc_gemm_wgrad"):
             getattr(lib, name).argtypes = [P, P, P, P, I64, I64, I64, P, P,
                                            ctypes.c_int]
@@ -99,11 +103,13 @@ def e4m3_encode(t) -> np.ndarray:
     return out
 
 
-def group_scale(amax: float):
+def group_scale(amax: float, pow2=False):
+    """(qscale, s) of a group with this amax; pow2 selects the power-of-two
+    scale form."""
     q = ctypes.c_float()
     s = ctypes.c_float()
-    _L().orc_group_scale(ctypes.c_float(amax), ctypes.byref(q),
-                         ctypes.byref(s))
+    fn = _L().orc_group_scale_pow2 if pow2 else _L().orc_group_scale
+    fn(ctypes.c_float(amax), ctypes.byref(q), ctypes.byref(s))
     return np.float32(q.value), np.float32(s.value)
 
 
@@ -122,33 +128,37 @@ def bf16_to_float(b) -> np.ndarray:
 
 # ---------------------------------------------------------------- quantisers
 
-def quantize_rowwise(x):
+def quantize_rowwise(x, pow2=False):
     x = _c(x, np.uint16)
     rows, cols = x.shape
     q = np.empty((rows, cols), np.uint8)
     s = np.empty((_cdiv(cols, 128), rows), np.float32)
-    rc = _L().orc_quantize_rowwise(_p(x), rows, cols, _p(q), _p(s))
+    fn = _L().orc_quantize_rowwise_pow2 if pow2 else _L().orc_quantize_rowwise
+    rc = fn(_p(x), rows, cols, _p(q), _p(s))
     assert rc == 0
     return q, s
 
 
-def quantize_colwise(x):
+def quantize_colwise(x, pow2=False):
     x = _c(x, np.uint16)
     rows, cols = x.shape
     q_t = np.empty((cols, rows), np.uint8)
     s_t = np.empty((_cdiv(rows, 128), cols), np.float32)
-    rc = _L().orc_quantize_colwise(_p(x), rows, cols, _p(q_t), _p(s_t))
+    fn = _L().orc_quantize_colwise_pow2 if pow2 else _L().orc_quantize_colwise
+    rc = fn(_p(x), rows, cols, _p(q_t), _p(s_t))
     assert rc == 0
     return q_t, s_t
 
 
-def quantize_weight_block(w, want_transposed=True):
+def quantize_weight_block(w, want_transposed=True, pow2=False):
     w = _c(w, np.uint16)
     n, k = w.shape
     q = np.empty((n, k), np.uint8)
     s = np.empty((_cdiv(n, 128), _cdiv(k, 128)), np.float32)
     q_t = np.empty((k, n), np.uint8) if want_transposed else None
-    rc = _L().orc_quantize_weight_block(_p(w), n, k, _p(q), _p(s), _p(q_t))
+    fn = _L().orc_quantize_weight_block_pow2 if pow2 else \
+        _L().orc_quantize_weight_block
+    rc = fn(_p(w), n, k, _p(q), _p(s), _p(q_t))
     assert rc == 0
     return q, s, q_t
 

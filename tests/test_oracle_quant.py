@@ -28,9 +28,9 @@ def f32_of(b):
     return (np.asarray(b, np.uint16).astype(np.uint32) << 16).view(np.float32)
 
 
-def _hand_groups():
+def _hand_groups(fname="quant_group_hand.txt"):
     rows = []
-    with open(os.path.join(GOLDEN, "quant_group_hand.txt")) as fh:
+    with open(os.path.join(GOLDEN, fname)) as fh:
         for line in fh:
             line = line.strip()
             if not line or line.startswith("#"):
@@ -157,3 +157,70 @@ def test_roundtrip_bound_rowwise_colwise_weight():
     qw, sw, _ = oracle.quantize_weight_block(w)
     full = np.repeat(np.repeat(sw, 128, axis=0), 128, axis=1)[:384, :640]
     _roundtrip_check(qw, full, f32_of(w))
+
+
+# ------------------------------------------------------------------ pow2 scales
+# Power-of-two reading (the form B200 tensor cores apply in hardware): s = 2^E,
+# E the smallest integer with 448 * 2^E >= amax, clamped to [-127, 127].
+
+@pytest.mark.parametrize("name,vals,fill,codes,sbits",
+                         _hand_groups("quant_pow2_hand.txt"))
+def test_pow2_hand_worked_group(name, vals, fill, codes, sbits):
+    g = np.full(128, fill, dtype=np.float32)
+    g[: len(vals)] = vals
+    q, s = oracle.quantize_rowwise(bf16_bits(g)[None, :], pow2=True)
+    assert q[0, : len(codes)].tolist() == codes, name
+    assert s.view(np.uint32)[0, 0] == sbits, (name, hex(s.view(np.uint32)[0, 0]))
+
+
+def _exact_pow2_exponent(amax):
+    """Smallest integer E with 448 * 2^E >= amax, by exact rational
+    arithmetic (independent of the oracle's binary64 search)."""
+    from fractions import Fraction
+    a = Fraction(float(amax))
+    e = 0
+    while Fraction(448) * Fraction(2) ** e < a:
+        e += 1
+    while Fraction(448) * Fraction(2) ** (e - 1) >= a:
+        e -= 1
+    return max(-127, min(127, e))
+
+
+def test_pow2_scale_is_the_smallest_covering_power_of_two():
+    rng = np.random.default_rng(7)
+    # bf16 magnitudes spread over the whole exponent range, plus ties at 448*2^k
+    bits = rng.integers(1, 0x7F80, 4000).astype(np.uint16)
+    amaxes = list(f32_of(bits)) + [448.0 * 2.0 ** k for k in range(-40, 40)]
+    for a in amaxes:
+        qscale, s = oracle.group_scale(float(a), pow2=True)
+        e = _exact_pow2_exponent(a)
+        assert float(s) == 2.0 ** e and float(qscale) == 2.0 ** -e, a
+
+
+def test_pow2_codes_match_an_independent_encoder():
+    import torch
+    x = S.bf16_normal((96, 640), 0, 111, 1.0, 1e-2, 50.0)
+    q, s = oracle.quantize_rowwise(x, pow2=True)
+    f = f32_of(x).reshape(96, 5, 128)
+    inv = (1.0 / s.T.astype(np.float64)).astype(np.float32)[:, :, None]
+    t = torch.from_numpy(np.ascontiguousarray(f * inv))   # exact: power of two
+    ref = t.to(torch.float8_e4m3fn).view(torch.uint8).numpy().reshape(96, 640)
+    assert np.array_equal(q, ref)
+    # the group's largest magnitude lands in (224, 448]
+    amax = np.abs(f).max(axis=2) / s.T
+    assert np.all((amax > 224) & (amax <= 448))
+
+
+def test_pow2_layouts_agree():
+    x = S.bf16_normal((272, 400), 0, 112, 1.0, 1e-3, 50.0)
+    q_r, s_r = oracle.quantize_rowwise(np.ascontiguousarray(x.T), pow2=True)
+    q_t, s_t = oracle.quantize_colwise(x, pow2=True)
+    assert np.array_equal(q_r, q_t) and np.array_equal(s_r, s_t)
+    w = S.bf16_normal((272, 400), 0, 113, **S.W_DIST)
+    qw, sw, qw_t = oracle.quantize_weight_block(w, pow2=True)
+    assert np.array_equal(qw_t, qw.T)
+    fw = np.abs(f32_of(w))
+    for nb in range(3):
+        for kb in range(4):
+            blk = fw[nb * 128:(nb + 1) * 128, kb * 128:(kb + 1) * 128]
+            assert float(sw[nb, kb]) == 2.0 ** _exact_pow2_exponent(blk.max())
