@@ -279,34 +279,37 @@ class LinearBuffers:
         self.qdy_t, self.sdy_t = e((n, m), u8), e((cd(m), n), f32)
         self.y, self.dx, self.dw = e((m, n), bf), e((m, k), bf), e((n, k), bf)
 
-    def ops(self, o, stream):
-        """[(kernel kind, algorithmic units, callable)] of this linear."""
+    def ops(self, o, stream, pow2=False):
+        """[(kernel kind, algorithmic units, callable)] of this linear; pow2
+        selects the power-of-two-scale quantisers and GEMMs."""
         m, k, n = TOKENS, self.k, self.n
         cd = lambda a: (a + 127) // 128  # noqa: E731
         wq_bytes = n * k * 2 + 2 * n * k + 4 * cd(n) * cd(k)
         xq_bytes = m * k * 2 + 2 * m * k + 4 * (m * cd(k) + cd(m) * k)
         dyq_bytes = m * n * 2 + 2 * m * n + 4 * (m * cd(n) + cd(m) * n)
         f = 2 * m * n * k
+        p2 = pow2
         return [
             ("quant_weight_block", wq_bytes,
              lambda: o.fp8bw_quantize_weight_block(self.w, self.qw, self.sw,
-                                                   self.qw_t, stream)),
+                                                   self.qw_t, stream, pow2=p2)),
             ("quant_rowcol", xq_bytes,
              lambda: o.fp8bw_quantize_colwise(self.x, self.qx_t, self.sx_t,
-                                              self.qx, self.sx, stream)),
+                                              self.qx, self.sx, stream,
+                                              pow2=p2)),
             ("gemm_block_scaled", f,
              lambda: o.fp8bw_gemm_fprop(self.qx, self.sx, self.qw, self.sw,
-                                        self.y, stream)),
+                                        self.y, stream, pow2=p2)),
             ("quant_rowcol", dyq_bytes,
              lambda: o.fp8bw_quantize_colwise(self.dy, self.qdy_t,
                                               self.sdy_t, self.qdy,
-                                              self.sdy, stream)),
+                                              self.sdy, stream, pow2=p2)),
             ("gemm_block_scaled", f,
              lambda: o.fp8bw_gemm_dgrad(self.qdy, self.sdy, self.qw_t, 1,
-                                        self.sw, self.dx, stream)),
+                                        self.sw, self.dx, stream, pow2=p2)),
             ("gemm_vector_scaled", f,
              lambda: o.fp8bw_gemm_wgrad(self.qdy_t, self.sdy_t, self.qx_t,
-                                        self.sx_t, self.dw, stream)),
+                                        self.sx_t, self.dw, stream, pow2=p2)),
         ]
 
 
@@ -340,11 +343,58 @@ def time_next_rows(o, bufs, stream, warmup, rounds):
     o.fp8bw_check_device_error(stream)
     ms = sum(e0.elapsed_time(e1) for r in ev for e0, e1 in r)
     flop = rounds * sum(f for f, _ in calls)
-    return {"wgrad_f32_accumulate": {
+    out = {"wgrad_f32_accumulate": {
         "achieved": flop / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
         "launches": rounds * len(calls), "avg_launch_ms": ms / (rounds * len(calls)),
         "what": "dW (fp32) += dY^T X for the QKV, O, gate/up and down "
                 "linears at M=%d, in turn; timed after the step" % TOKENS}}
+
+    # The whole step again with power-of-two scales (quantisers and GEMMs on
+    # the tensor cores' UE8M0 block scaling), same buffers and order.
+    step = []
+    for _layer in range(LAYERS):
+        for b in bufs:
+            step.extend(b.ops(o, stream, pow2=True))
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            for _, _, fn in step:
+                fn()
+    torch.cuda.synchronize()
+    steps = 3
+    evs = [[(torch.cuda.Event(enable_timing=True),
+             torch.cuda.Event(enable_timing=True)) for _ in step]
+           for _ in range(steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for s in range(steps):
+            for (_, _, fn), (e0, e1) in zip(step, evs[s]):
+                e0.record(stream)
+                fn()
+                e1.record(stream)
+        t1.record(stream)
+    torch.cuda.synchronize()
+    o.fp8bw_check_device_error(stream)
+    step_ms = t0.elapsed_time(t1) / steps
+    kinds_ = {}
+    for s in range(steps):
+        for (kk, units, _), (e0, e1) in zip(step, evs[s]):
+            d = kinds_.setdefault(kk, [0.0, 0])
+            d[0] += e0.elapsed_time(e1)
+            d[1] += units
+    gflop = sum(u for kk, u, _ in step if kk.startswith("gemm"))
+    out["pow2_step"] = {
+        "achieved": gflop / (step_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "ms_per_step": step_ms, "steps": steps,
+        "breakdown": {kk: (u / (ms_ * 1e-3) / 1e12 if kk.startswith("gemm")
+                           else u / (ms_ * 1e-3) / 1e9)
+                      for kk, (ms_, u) in kinds_.items()},
+        "breakdown_units": "gemm_*: TFLOP/s, quant_*: GB/s",
+        "what": "the same 28-layer step with power-of-two scales (s = 2^E, "
+                "the smallest E with 448*2^E >= amax) applied by the tensor "
+                "cores' UE8M0 block scaling; timed after the step"}
+    return out
 
 
 class ClockSampler:
@@ -586,7 +636,8 @@ def run_gpu(args):
 
     if next_rows is not None:
         for d in next_rows.values():
-            d["frac_of_fp8_peak"] = d["achieved"] / fp8_sustained
+            if d.get("unit") == "TFLOP/s":
+                d["frac_of_fp8_peak"] = d["achieved"] / fp8_sustained
     value = weak_scaling_value(world, flops, ms * 1e-3) / 1e12
     line = {
         "metric": METRIC,

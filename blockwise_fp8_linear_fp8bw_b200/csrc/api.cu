@@ -13,6 +13,7 @@
 
 #include "common.cuh"
 #include "gemm_pair.cuh"
+#include "gemm_pow2.cuh"
 #include "quant.cuh"
 
 #ifndef GEMM_BN_BLOCK
@@ -171,6 +172,7 @@ struct GemmProblem {
   int64_t sbj, sbc;
   void* out;         // [mo][no]: bf16 (kOutBf16) or fp32
   int out_mode;      // gemm::kOutBf16 / kOutF32 / kOutF32Add
+  bool pow2;         // power-of-two scales on the hardware block-scaled MMA
 };
 
 // CTA-pair kernel: 256 x 256 output tiles on clusters of two CTAs.
@@ -249,6 +251,68 @@ int launch_gemm_pair(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t s
   return cudaGetLastError() == cudaSuccess ? FP8BW_OK : FP8BW_ERR_LAUNCH;
 }
 
+// Power-of-two-scale kernel (hardware block scaling), same problem description.
+template <bool VEC_B, bool B_MN>
+int launch_gemm_pow2(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t stream) {
+  using L = gemm_pow2::Layout;
+  auto kernel = gemm_pow2::blockwise_gemm_pow2_kernel<VEC_B, B_MN>;
+  static std::once_flag once;
+  static int prep_status = FP8BW_OK;
+  static int max_clusters = 0;
+  std::call_once(once, [&]() {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) !=
+        cudaSuccess) {
+      prep_status = FP8BW_ERR_LAUNCH;
+      return;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * dev.sm_count, 1, 1);
+    cfg.blockDim = dim3(gemm_pow2::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = L::kAlloc;
+    cudaLaunchAttribute attr_cl;
+    attr_cl.id = cudaLaunchAttributeClusterDimension;
+    attr_cl.val.clusterDim.x = 2;
+    attr_cl.val.clusterDim.y = 1;
+    attr_cl.val.clusterDim.z = 1;
+    cfg.attrs = &attr_cl;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&max_clusters, kernel, &cfg) != cudaSuccess ||
+        max_clusters < 1)
+      prep_status = FP8BW_ERR_LAUNCH;
+  });
+  if (prep_status != FP8BW_OK) return prep_status;
+
+  CUtensorMap tm_a, tm_b, tm_out;
+  int st = encode_u8_2d(&tm_a, p.a, static_cast<uint64_t>(p.kc), static_cast<uint64_t>(p.mo),
+                        gemm_pow2::BM);
+  if (st != FP8BW_OK) return st;
+  if (B_MN)
+    st = encode_u8_2d(&tm_b, p.b, static_cast<uint64_t>(p.no), static_cast<uint64_t>(p.kc), 128);
+  else
+    st = encode_u8_2d(&tm_b, p.b, static_cast<uint64_t>(p.kc), static_cast<uint64_t>(p.no),
+                      gemm_pow2::BN / 2);
+  if (st != FP8BW_OK) return st;
+  st = encode_bf16_out(&tm_out, p.out, static_cast<uint64_t>(p.no), static_cast<uint64_t>(p.mo));
+  if (st != FP8BW_OK) return st;
+
+  gemm_pow2::Args g;
+  g.mo = static_cast<int>(p.mo);
+  g.no = static_cast<int>(p.no);
+  g.kc = static_cast<int>(p.kc);
+  g.tiles_m = static_cast<int>(cdiv(p.mo, 2 * gemm_pow2::BM));
+  g.tiles_n = static_cast<int>(cdiv(p.no, gemm_pow2::BN));
+  g.chunks = static_cast<int>(cdiv(p.kc, gemm_pow2::BK));
+  g.sa = p.sa;
+  g.sb = p.sb;
+  g.sbj = p.sbj;
+  g.sbc = p.sbc;
+  g.nblk = static_cast<int>(cdiv(p.no, 128));
+  const int64_t tiles = static_cast<int64_t>(g.tiles_m) * g.tiles_n;
+  const int clusters = static_cast<int>(std::min<int64_t>(tiles, max_clusters));
+  kernel<<<2 * clusters, gemm_pow2::kThreads, L::kAlloc, stream>>>(tm_a, tm_b, tm_out, g);
+  return cudaGetLastError() == cudaSuccess ? FP8BW_OK : FP8BW_ERR_LAUNCH;
+}
+
 int run_gemm(const GemmProblem& p, cudaStream_t stream) {
   DeviceInfo dev;
   int st = current_device_info(&dev);
@@ -264,6 +328,12 @@ int run_gemm(const GemmProblem& p, cudaStream_t stream) {
                : FP8BW_ERR_CUDA;
   }
   if (cdiv(p.mo, 256) * cdiv(p.no, 256) > (int64_t(1) << 30)) return FP8BW_ERR_SHAPE;
+  if (p.pow2) {
+    if (p.out_mode != gemm::kOutBf16) return FP8BW_ERR_LAUNCH;
+    if (p.vec_b) return launch_gemm_pow2<true, false>(p, dev, stream);
+    if (p.b_mn) return launch_gemm_pow2<false, true>(p, dev, stream);
+    return launch_gemm_pow2<false, false>(p, dev, stream);
+  }
   if (p.vec_b && p.out_mode == gemm::kOutF32)
     return launch_gemm_pair<GEMM_BN_VEC, true, false, gemm::kOutF32>(p, dev, stream);
   if (p.vec_b && p.out_mode == gemm::kOutF32Add)
@@ -281,7 +351,7 @@ using namespace fp8bw;
 
 extern "C" {
 
-int fp8bw_version(void) { return 101; }
+int fp8bw_version(void) { return 102; }
 
 const char* fp8bw_status_string(int status) {
   switch (status) {
@@ -294,12 +364,18 @@ const char* fp8bw_status_string(int status) {
     case FP8BW_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait expired";
     case FP8BW_ERR_CUDA: return "a CUDA runtime or driver call failed";
     case FP8BW_ERR_ALIAS: return "an output buffer overlaps an input buffer";
+    case FP8BW_ERR_SCALE:
+      return "a power-of-two GEMM was given a scale that is not a power of two";
     default: return "unknown status";
   }
 }
 
-int fp8bw_quantize_rowwise(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* q, float* s,
-                           void* stream) {
+}  // extern "C"
+
+namespace {
+
+int quantize_rowwise(bool pow2, const uint16_t* x, int64_t rows, int64_t cols, uint8_t* q,
+                     float* s, void* stream) {
   if (!dim_ok(rows) || !dim_ok(cols) || cdiv(rows, 128) > 65535) return FP8BW_ERR_SHAPE;
   if (missing(x, rows * cols) || missing(q, rows * cols) || missing(s, cdiv(cols, 128) * rows))
     return FP8BW_ERR_NULL;
@@ -311,12 +387,12 @@ int fp8bw_quantize_rowwise(const uint16_t* x, int64_t rows, int64_t cols, uint8_
   int st = current_device_info(&dev);
   if (st != FP8BW_OK) return st;
   if (rows == 0 || cols == 0) return FP8BW_OK;
-  return launch_quantize(kModeRow, x, rows, cols, q, s, nullptr, nullptr, nullptr, dev.sm_count,
+  return launch_quantize(kModeRow, pow2, x, rows, cols, q, s, nullptr, nullptr, nullptr, dev.sm_count,
                          static_cast<cudaStream_t>(stream));
 }
 
-int fp8bw_quantize_colwise(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* q_t,
-                           float* s_t, uint8_t* q_row, float* s_row, void* stream) {
+int quantize_colwise(bool pow2, const uint16_t* x, int64_t rows, int64_t cols, uint8_t* q_t,
+                     float* s_t, uint8_t* q_row, float* s_row, void* stream) {
   if (!dim_ok(rows) || !dim_ok(cols) || cdiv(rows, 128) > 65535) return FP8BW_ERR_SHAPE;
   if (missing(x, rows * cols) || missing(q_t, rows * cols) || missing(s_t, cdiv(rows, 128) * cols))
     return FP8BW_ERR_NULL;
@@ -335,12 +411,12 @@ int fp8bw_quantize_colwise(const uint16_t* x, int64_t rows, int64_t cols, uint8_
   if (st != FP8BW_OK) return st;
   if (rows == 0 || cols == 0) return FP8BW_OK;
   const int mode = q_row ? kModeRowCol : kModeCol;
-  return launch_quantize(mode, x, rows, cols, q_row, s_row, q_t, s_t, nullptr, dev.sm_count,
+  return launch_quantize(mode, pow2, x, rows, cols, q_row, s_row, q_t, s_t, nullptr, dev.sm_count,
                          static_cast<cudaStream_t>(stream));
 }
 
-int fp8bw_quantize_weight_block(const uint16_t* w, int64_t n, int64_t k, uint8_t* q, float* s,
-                                uint8_t* q_t, void* stream) {
+int quantize_weight_block(bool pow2, const uint16_t* w, int64_t n, int64_t k, uint8_t* q,
+                          float* s, uint8_t* q_t, void* stream) {
   if (!dim_ok(n) || !dim_ok(k) || cdiv(n, 128) > 65535) return FP8BW_ERR_SHAPE;
   if (missing(w, n * k) || missing(q, n * k) || missing(s, cdiv(n, 128) * cdiv(k, 128)))
     return FP8BW_ERR_NULL;
@@ -353,12 +429,50 @@ int fp8bw_quantize_weight_block(const uint16_t* w, int64_t n, int64_t k, uint8_t
   int st = current_device_info(&dev);
   if (st != FP8BW_OK) return st;
   if (n == 0 || k == 0) return FP8BW_OK;
-  return launch_quantize(kModeBlock, w, n, k, q, nullptr, q_t, nullptr, s, dev.sm_count,
+  return launch_quantize(kModeBlock, pow2, w, n, k, q, nullptr, q_t, nullptr, s, dev.sm_count,
                          static_cast<cudaStream_t>(stream));
 }
 
-int fp8bw_gemm_fprop(const uint8_t* qx, const float* sx, const uint8_t* qw, const float* sw,
-                     int64_t m, int64_t n, int64_t k, uint16_t* y, void* stream) {
+}  // namespace
+
+extern "C" {
+
+int fp8bw_quantize_rowwise(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* q, float* s,
+                           void* stream) {
+  return quantize_rowwise(false, x, rows, cols, q, s, stream);
+}
+
+int fp8bw_quantize_colwise(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* q_t,
+                           float* s_t, uint8_t* q_row, float* s_row, void* stream) {
+  return quantize_colwise(false, x, rows, cols, q_t, s_t, q_row, s_row, stream);
+}
+
+int fp8bw_quantize_weight_block(const uint16_t* w, int64_t n, int64_t k, uint8_t* q, float* s,
+                                uint8_t* q_t, void* stream) {
+  return quantize_weight_block(false, w, n, k, q, s, q_t, stream);
+}
+
+int fp8bw_quantize_rowwise_pow2(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* q,
+                                float* s, void* stream) {
+  return quantize_rowwise(true, x, rows, cols, q, s, stream);
+}
+
+int fp8bw_quantize_colwise_pow2(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* q_t,
+                                float* s_t, uint8_t* q_row, float* s_row, void* stream) {
+  return quantize_colwise(true, x, rows, cols, q_t, s_t, q_row, s_row, stream);
+}
+
+int fp8bw_quantize_weight_block_pow2(const uint16_t* w, int64_t n, int64_t k, uint8_t* q,
+                                     float* s, uint8_t* q_t, void* stream) {
+  return quantize_weight_block(true, w, n, k, q, s, q_t, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+int gemm_fprop(bool pow2, const uint8_t* qx, const float* sx, const uint8_t* qw, const float* sw,
+               int64_t m, int64_t n, int64_t k, uint16_t* y, void* stream) {
   if (!dim_ok(m) || !dim_ok(n) || !dim_ok(k)) return FP8BW_ERR_SHAPE;
   if (missing(qx, m * k) || missing(sx, cdiv(k, 128) * m) || missing(qw, n * k) ||
       missing(sw, cdiv(n, 128) * cdiv(k, 128)) || missing(y, m * n))
@@ -382,12 +496,13 @@ int fp8bw_gemm_fprop(const uint8_t* qx, const float* sx, const uint8_t* qw, cons
   p.sbj = cdiv(k, 128);  // sW[n/128][c]
   p.sbc = 1;
   p.out = y;
+  p.pow2 = pow2;
   return run_gemm(p, static_cast<cudaStream_t>(stream));
 }
 
-int fp8bw_gemm_dgrad(const uint8_t* qdy, const float* sdy, const uint8_t* qw,
-                     int qw_is_transposed, const float* sw, int64_t m, int64_t n, int64_t k,
-                     uint16_t* dx, void* stream) {
+int gemm_dgrad(bool pow2, const uint8_t* qdy, const float* sdy, const uint8_t* qw,
+               int qw_is_transposed, const float* sw, int64_t m, int64_t n, int64_t k,
+               uint16_t* dx, void* stream) {
   if (!dim_ok(m) || !dim_ok(n) || !dim_ok(k)) return FP8BW_ERR_SHAPE;
   if (missing(qdy, m * n) || missing(sdy, cdiv(n, 128) * m) || missing(qw, n * k) ||
       missing(sw, cdiv(n, 128) * cdiv(k, 128)) || missing(dx, m * k))
@@ -411,7 +526,34 @@ int fp8bw_gemm_dgrad(const uint8_t* qdy, const float* sdy, const uint8_t* qw,
   p.sbj = 1;             // sW[c][k/128]
   p.sbc = cdiv(k, 128);
   p.out = dx;
+  p.pow2 = pow2;
   return run_gemm(p, static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+int fp8bw_gemm_fprop(const uint8_t* qx, const float* sx, const uint8_t* qw, const float* sw,
+                     int64_t m, int64_t n, int64_t k, uint16_t* y, void* stream) {
+  return gemm_fprop(false, qx, sx, qw, sw, m, n, k, y, stream);
+}
+
+int fp8bw_gemm_dgrad(const uint8_t* qdy, const float* sdy, const uint8_t* qw,
+                     int qw_is_transposed, const float* sw, int64_t m, int64_t n, int64_t k,
+                     uint16_t* dx, void* stream) {
+  return gemm_dgrad(false, qdy, sdy, qw, qw_is_transposed, sw, m, n, k, dx, stream);
+}
+
+int fp8bw_gemm_fprop_pow2(const uint8_t* qx, const float* sx, const uint8_t* qw, const float* sw,
+                          int64_t m, int64_t n, int64_t k, uint16_t* y, void* stream) {
+  return gemm_fprop(true, qx, sx, qw, sw, m, n, k, y, stream);
+}
+
+int fp8bw_gemm_dgrad_pow2(const uint8_t* qdy, const float* sdy, const uint8_t* qw,
+                          int qw_is_transposed, const float* sw, int64_t m, int64_t n,
+                          int64_t k, uint16_t* dx, void* stream) {
+  return gemm_dgrad(true, qdy, sdy, qw, qw_is_transposed, sw, m, n, k, dx, stream);
 }
 
 }  // extern "C"
@@ -420,7 +562,7 @@ namespace {
 
 int wgrad_common(const uint8_t* qdy_t, const float* sdy_t, const uint8_t* qx_t,
                  const float* sx_t, int64_t m, int64_t n, int64_t k, void* dw, int out_mode,
-                 void* stream) {
+                 bool pow2, void* stream) {
   if (!dim_ok(m) || !dim_ok(n) || !dim_ok(k)) return FP8BW_ERR_SHAPE;
   if (missing(qdy_t, n * m) || missing(sdy_t, cdiv(m, 128) * n) || missing(qx_t, k * m) ||
       missing(sx_t, cdiv(m, 128) * k) || missing(dw, n * k))
@@ -447,6 +589,7 @@ int wgrad_common(const uint8_t* qdy_t, const float* sdy_t, const uint8_t* qx_t,
   p.sbc = 0;
   p.out = dw;
   p.out_mode = out_mode;
+  p.pow2 = pow2;
   return run_gemm(p, static_cast<cudaStream_t>(stream));
 }
 
@@ -457,14 +600,20 @@ extern "C" {
 int fp8bw_gemm_wgrad(const uint8_t* qdy_t, const float* sdy_t, const uint8_t* qx_t,
                      const float* sx_t, int64_t m, int64_t n, int64_t k, uint16_t* dw,
                      void* stream) {
-  return wgrad_common(qdy_t, sdy_t, qx_t, sx_t, m, n, k, dw, gemm::kOutBf16, stream);
+  return wgrad_common(qdy_t, sdy_t, qx_t, sx_t, m, n, k, dw, gemm::kOutBf16, false, stream);
+}
+
+int fp8bw_gemm_wgrad_pow2(const uint8_t* qdy_t, const float* sdy_t, const uint8_t* qx_t,
+                          const float* sx_t, int64_t m, int64_t n, int64_t k, uint16_t* dw,
+                          void* stream) {
+  return wgrad_common(qdy_t, sdy_t, qx_t, sx_t, m, n, k, dw, gemm::kOutBf16, true, stream);
 }
 
 int fp8bw_gemm_wgrad_f32(const uint8_t* qdy_t, const float* sdy_t, const uint8_t* qx_t,
                          const float* sx_t, int64_t m, int64_t n, int64_t k, float* dw,
                          int accumulate, void* stream) {
   return wgrad_common(qdy_t, sdy_t, qx_t, sx_t, m, n, k, dw,
-                      accumulate ? gemm::kOutF32Add : gemm::kOutF32, stream);
+                      accumulate ? gemm::kOutF32Add : gemm::kOutF32, false, stream);
 }
 
 int fp8bw_check_device_error(void* stream) {
@@ -476,7 +625,9 @@ int fp8bw_check_device_error(void* stream) {
   if (v != 0u &&
       cudaMemcpyToSymbol(fp8bw::g_device_error, &zero, sizeof zero) != cudaSuccess)
     return FP8BW_ERR_CUDA;
-  return v != 0u ? FP8BW_ERR_DEVICE_TIMEOUT : FP8BW_OK;
+  if (v == 0u) return FP8BW_OK;
+  return (v & ~static_cast<uint32_t>(kErrScaleNotPow2)) != 0u ? FP8BW_ERR_DEVICE_TIMEOUT
+                                                              : FP8BW_ERR_SCALE;
 }
 
 }  // extern "C"

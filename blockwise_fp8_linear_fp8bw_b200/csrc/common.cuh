@@ -19,6 +19,7 @@ enum : uint32_t {
   kErrTimeoutMma = 2u,
   kErrTimeoutEpi = 4u,
   kErrTimeoutScale = 8u,
+  kErrScaleNotPow2 = 16u,   // a power-of-two GEMM was given another scale
 };
 
 // Defined once: the library is a single translation unit.
@@ -465,6 +466,55 @@ __host__ __device__ constexpr uint32_t idesc_e4m3(int m, int n, bool b_mn_major)
   return (1u << 4) | ((b_mn_major ? 1u : 0u) << 16) |
          (static_cast<uint32_t>(n >> 3) << 17) |
          (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+// ---------------------------------------------------------------------------
+// Block-scaled MMA (kind::mxf8f6f4 with UE8M0 scale factors in TMEM)
+// ---------------------------------------------------------------------------
+
+// Instruction descriptor of kind::mxf8f6f4.block_scale: A and B E4M3 (format
+// 0 at bits 7-9 and 10-12), A K-major, B K-major or MN-major (bit 16), N >> 3
+// at bits 17-22, scale format UE8M0 (bit 23 = 1), M >> 4 at bits 24-28, and
+// the byte of the 32-bit scale-factor word to use for B (bits 4-5) and A
+// (bits 29-30). The accumulator is always fp32.
+__host__ __device__ constexpr uint32_t idesc_e4m3_ue8m0(int m, int n, bool b_mn_major,
+                                                        uint32_t sf_byte) {
+  return ((sf_byte & 3u) << 4) | ((b_mn_major ? 1u : 0u) << 16) |
+         (static_cast<uint32_t>(n >> 3) << 17) | (1u << 23) |
+         (static_cast<uint32_t>(m >> 4) << 24) | ((sf_byte & 3u) << 29);
+}
+
+// D (+)= (A * 2^SFA) x (B * 2^SFB)^T over K = 32, issued for the CTA pair;
+// sfa / sfb are the TMEM addresses of the scale-factor columns.
+__device__ __forceinline__ void mma_mx_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], "
+      "p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Shared -> TMEM copy of 32 rows x 128 bits, replicated into the four 32-lane
+// quarters of TMEM, for both CTAs of the pair (each from its own shared
+// memory at the same offset). `desc` describes the 512-byte source.
+__device__ __forceinline__ void tmem_cp_32x128_x4_pair(uint32_t taddr, uint64_t desc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc)
+               : "memory");
+}
+
+// Shared-memory descriptor of 32 contiguous 16-byte rows (no swizzle, K-major:
+// 8-row core matrices 128 bytes apart).
+__device__ __forceinline__ uint64_t desc_rows16(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(128u >> 4) << 16;
+  d |= static_cast<uint64_t>(128u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  return d;
 }
 
 }  // namespace fp8bw

@@ -94,6 +94,35 @@ __device__ __forceinline__ void group_scale(float amax, float& qscale,
   }
 }
 
+// Power-of-two form: s = 2^E with E the smallest integer such that
+// 448 * 2^E >= amax, clamped below at -127 (a finite bf16 amax <= 3.39e38
+// keeps E <= 120, so qscale = 2^-E is always a normal float). With
+// amax = (1 + f) * 2^(ef - 127): E = ef - 135 when 1 + f <= 1.75 (448 =
+// 1.75 * 2^8), else ef - 134; a subnormal amax gives E = -127. All integer
+// work on the bits, so the result is exact.
+__device__ __forceinline__ void group_scale_pow2(float amax, float& qscale, float& s) {
+  if (amax == 0.0f || !isfinite(amax)) {
+    qscale = 1.0f;
+    s = 1.0f;
+    return;
+  }
+  const uint32_t b = __float_as_uint(amax);
+  const int ef = static_cast<int>(b >> 23);
+  int e = ef == 0 ? -127 : ef - 135 + ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+  e = max(-127, min(120, e));
+  s = e >= -126 ? __uint_as_float(static_cast<uint32_t>(e + 127) << 23)
+                : __uint_as_float(0x00400000u);   // 2^-127, a subnormal
+  qscale = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+}
+
+template <bool POW2>
+__device__ __forceinline__ void scale_of(float amax, float& qscale, float& s) {
+  if constexpr (POW2)
+    group_scale_pow2(amax, qscale, s);
+  else
+    group_scale(amax, qscale, s);
+}
+
 // |x| of two packed bf16 values (clears both sign bits; exact).
 __device__ __forceinline__ uint32_t abs_bf16x2(uint32_t w) { return w & 0x7FFF7FFFu; }
 
@@ -138,7 +167,7 @@ __device__ __forceinline__ int t_unit_offset(int k, int u) {
   return k * kQTile + ((u ^ (k >> 3)) & 15) * 8;
 }
 
-template <int MODE>
+template <int MODE, bool POW2>
 __global__ void __launch_bounds__(kQThreads, 2)
     quant_tile_kernel(const __grid_constant__ CUtensorMap tm_x, const QuantArgs a) {
   extern __shared__ uint8_t qsmem_raw[];
@@ -238,7 +267,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
 #pragma unroll
       for (int w = 1; w < kQThreads / 32; ++w) amax = fmaxf(amax, blk[w]);
       float qs, s;
-      group_scale(amax, qs, s);
+      scale_of<POW2>(amax, qs, s);
       if (t == 0) a.s_block[static_cast<int64_t>(tr) * a.tiles_c + tc] = s;
       if (cvalid && rvalid) {
 #pragma unroll
@@ -280,7 +309,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
           if ((cg & 7) == p) my_amax = am;
         }
         float my_qs, my_s;
-        group_scale(my_amax, my_qs, my_s);
+        scale_of<POW2>(my_amax, my_qs, my_s);
         if (cg < 8) srow_s[rb * 8 + cg] = my_s;
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
@@ -317,7 +346,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
 #pragma unroll
           for (int w = 1; w < kQThreads / 32; ++w) m = fmaxf(m, red[w][t]);
           float qs, s;
-          group_scale(m, qs, s);
+          scale_of<POW2>(m, qs, s);
           colq[t] = qs;
           const int64_t col = static_cast<int64_t>(tc) * kQTile + t;
           if (col < cols) a.s_col[static_cast<int64_t>(tr) * cols + col] = s;
@@ -390,9 +419,9 @@ __global__ void __launch_bounds__(kQThreads, 2)
 int encode_bf16_in(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows);
 
 // Launchers (shapes and pointers already validated by the C ABI layer).
-int launch_quantize(int mode, const uint16_t* x, int64_t rows, int64_t cols, uint8_t* q_row,
-                    float* s_row, uint8_t* q_col, float* s_col, float* s_block, int sm_count,
-                    cudaStream_t stream) {
+int launch_quantize(int mode, bool pow2, const uint16_t* x, int64_t rows, int64_t cols,
+                    uint8_t* q_row, float* s_row, uint8_t* q_col, float* s_col, float* s_block,
+                    int sm_count, cudaStream_t stream) {
   QuantArgs a{rows, cols, static_cast<int>((rows + kQTile - 1) / kQTile),
               static_cast<int>((cols + kQTile - 1) / kQTile), q_row, s_row, q_col, s_col, s_block};
   CUtensorMap tm;
@@ -401,8 +430,11 @@ int launch_quantize(int mode, const uint16_t* x, int64_t rows, int64_t cols, uin
   const int tiles = a.tiles_r * a.tiles_c;
   const int grid = tiles < 2 * sm_count ? tiles : 2 * sm_count;
   using Kernel = void (*)(CUtensorMap, QuantArgs);
-  static const Kernel kernels[4] = {quant_tile_kernel<kModeRow>, quant_tile_kernel<kModeCol>,
-                                    quant_tile_kernel<kModeRowCol>, quant_tile_kernel<kModeBlock>};
+  static const Kernel kernels[8] = {
+      quant_tile_kernel<kModeRow, false>,    quant_tile_kernel<kModeCol, false>,
+      quant_tile_kernel<kModeRowCol, false>, quant_tile_kernel<kModeBlock, false>,
+      quant_tile_kernel<kModeRow, true>,     quant_tile_kernel<kModeCol, true>,
+      quant_tile_kernel<kModeRowCol, true>,  quant_tile_kernel<kModeBlock, true>};
   static std::once_flag once;
   static int prep = FP8BW_OK;
   std::call_once(once, [&]() {
@@ -412,7 +444,7 @@ int launch_quantize(int mode, const uint16_t* x, int64_t rows, int64_t cols, uin
         prep = FP8BW_ERR_LAUNCH;
   });
   if (prep != FP8BW_OK) return prep;
-  const Kernel kernel = kernels[mode >= 0 && mode < 4 ? mode : kModeBlock];
+  const Kernel kernel = kernels[(mode >= 0 && mode < 4 ? mode : kModeBlock) + (pow2 ? 4 : 0)];
   kernel<<<grid, kQThreads, QuantSmem::kAlloc, stream>>>(tm, a);
   return cudaGetLastError() == cudaSuccess ? FP8BW_OK : FP8BW_ERR_LAUNCH;
 }

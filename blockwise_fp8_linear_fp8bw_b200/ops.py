@@ -18,6 +18,7 @@ FP8BW_ERR_LAUNCH = -5
 FP8BW_ERR_DEVICE_TIMEOUT = -6
 FP8BW_ERR_CUDA = -7
 FP8BW_ERR_ALIAS = -8
+FP8BW_ERR_SCALE = -9
 
 _lib = _native.load()
 
@@ -60,19 +61,26 @@ def _cdiv(a, b):
     return (a + b - 1) // b
 
 
+def _fn(name, pow2):
+    """The entry point, or its power-of-two-scale variant."""
+    return name + "_pow2" if pow2 else name
+
+
 # ----------------------------------------------------------- raw entry points
 
-def fp8bw_quantize_rowwise(x, q, s, stream=None):
+def fp8bw_quantize_rowwise(x, q, s, stream=None, pow2=False):
     rows, cols = x.shape
     _expect(x, torch.bfloat16, (rows, cols), "x")
     _expect(q, torch.uint8, (rows, cols), "q")
     _expect(s, torch.float32, (_cdiv(cols, 128), rows), "s")
-    _check(_lib.fp8bw_quantize_rowwise(_ptr(x), rows, cols, _ptr(q), _ptr(s),
-                                       _stream(stream)),
-           "fp8bw_quantize_rowwise")
+    name = _fn('fp8bw_quantize_rowwise', pow2)
+    _check(getattr(_lib, name)(_ptr(x), rows, cols, _ptr(q), _ptr(s),
+                               _stream(stream)),
+           name)
 
 
-def fp8bw_quantize_colwise(x, q_t, s_t, q_row=None, s_row=None, stream=None):
+def fp8bw_quantize_colwise(x, q_t, s_t, q_row=None, s_row=None, stream=None,
+                           pow2=False):
     rows, cols = x.shape
     _expect(x, torch.bfloat16, (rows, cols), "x")
     _expect(q_t, torch.uint8, (cols, rows), "q_t")
@@ -80,60 +88,67 @@ def fp8bw_quantize_colwise(x, q_t, s_t, q_row=None, s_row=None, stream=None):
     if q_row is not None:
         _expect(q_row, torch.uint8, (rows, cols), "q_row")
         _expect(s_row, torch.float32, (_cdiv(cols, 128), rows), "s_row")
-    _check(_lib.fp8bw_quantize_colwise(_ptr(x), rows, cols, _ptr(q_t),
-                                       _ptr(s_t), _ptr(q_row), _ptr(s_row),
-                                       _stream(stream)),
-           "fp8bw_quantize_colwise")
+    name = _fn('fp8bw_quantize_colwise', pow2)
+    _check(getattr(_lib, name)(_ptr(x), rows, cols, _ptr(q_t),
+                               _ptr(s_t), _ptr(q_row), _ptr(s_row),
+                               _stream(stream)),
+           name)
 
 
-def fp8bw_quantize_weight_block(w, q, s, q_t=None, stream=None):
+def fp8bw_quantize_weight_block(w, q, s, q_t=None, stream=None,
+                                pow2=False):
     n, k = w.shape
     _expect(w, torch.bfloat16, (n, k), "w")
     _expect(q, torch.uint8, (n, k), "q")
     _expect(s, torch.float32, (_cdiv(n, 128), _cdiv(k, 128)), "s")
     if q_t is not None:
         _expect(q_t, torch.uint8, (k, n), "q_t")
-    _check(_lib.fp8bw_quantize_weight_block(_ptr(w), n, k, _ptr(q), _ptr(s),
-                                            _ptr(q_t), _stream(stream)),
-           "fp8bw_quantize_weight_block")
+    name = _fn('fp8bw_quantize_weight_block', pow2)
+    _check(getattr(_lib, name)(_ptr(w), n, k, _ptr(q), _ptr(s),
+                               _ptr(q_t), _stream(stream)),
+           name)
 
 
-def fp8bw_gemm_fprop(qx, sx, qw, sw, y, stream=None):
+def fp8bw_gemm_fprop(qx, sx, qw, sw, y, stream=None, pow2=False):
     m, k = qx.shape
     n = qw.shape[0]
     _expect(qw, torch.uint8, (n, k), "qw")
     _expect(sx, torch.float32, (_cdiv(k, 128), m), "sx")
     _expect(sw, torch.float32, (_cdiv(n, 128), _cdiv(k, 128)), "sw")
     _expect(y, torch.bfloat16, (m, n), "y")
-    _check(_lib.fp8bw_gemm_fprop(_ptr(qx), _ptr(sx), _ptr(qw), _ptr(sw), m, n,
-                                 k, _ptr(y), _stream(stream)),
-           "fp8bw_gemm_fprop")
+    name = _fn('fp8bw_gemm_fprop', pow2)
+    _check(getattr(_lib, name)(_ptr(qx), _ptr(sx), _ptr(qw), _ptr(sw), m, n,
+                               k, _ptr(y), _stream(stream)),
+           name)
 
 
-def fp8bw_gemm_dgrad(qdy, sdy, qw, qw_is_transposed, sw, dx, stream=None):
+def fp8bw_gemm_dgrad(qdy, sdy, qw, qw_is_transposed, sw, dx, stream=None,
+                     pow2=False):
     m, n = qdy.shape
     k = qw.shape[0] if qw_is_transposed else qw.shape[1]
     _expect(qw, torch.uint8, (k, n) if qw_is_transposed else (n, k), "qw")
     _expect(sdy, torch.float32, (_cdiv(n, 128), m), "sdy")
     _expect(sw, torch.float32, (_cdiv(n, 128), _cdiv(k, 128)), "sw")
     _expect(dx, torch.bfloat16, (m, k), "dx")
-    _check(_lib.fp8bw_gemm_dgrad(_ptr(qdy), _ptr(sdy), _ptr(qw),
-                                 1 if qw_is_transposed else 0, _ptr(sw), m, n,
-                                 k, _ptr(dx), _stream(stream)),
-           "fp8bw_gemm_dgrad")
+    name = _fn('fp8bw_gemm_dgrad', pow2)
+    _check(getattr(_lib, name)(_ptr(qdy), _ptr(sdy), _ptr(qw),
+                               1 if qw_is_transposed else 0, _ptr(sw), m, n,
+                               k, _ptr(dx), _stream(stream)),
+           name)
 
 
-def fp8bw_gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t, dw, stream=None):
+def fp8bw_gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t, dw, stream=None, pow2=False):
     n, m = qdy_t.shape
     k = qx_t.shape[0]
     _expect(qx_t, torch.uint8, (k, m), "qx_t")
     _expect(sdy_t, torch.float32, (_cdiv(m, 128), n), "sdy_t")
     _expect(sx_t, torch.float32, (_cdiv(m, 128), k), "sx_t")
     _expect(dw, torch.bfloat16, (n, k), "dw")
-    _check(_lib.fp8bw_gemm_wgrad(_ptr(qdy_t), _ptr(sdy_t), _ptr(qx_t),
-                                 _ptr(sx_t), m, n, k, _ptr(dw),
-                                 _stream(stream)),
-           "fp8bw_gemm_wgrad")
+    name = _fn('fp8bw_gemm_wgrad', pow2)
+    _check(getattr(_lib, name)(_ptr(qdy_t), _ptr(sdy_t), _ptr(qx_t),
+                               _ptr(sx_t), m, n, k, _ptr(dw),
+                               _stream(stream)),
+           name)
 
 
 def fp8bw_gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, dw, accumulate=False,
@@ -157,16 +172,16 @@ def fp8bw_check_device_error(stream=None):
 
 # ----------------------------------------------------------- allocating helpers
 
-def quantize_rowwise(x, stream=None):
+def quantize_rowwise(x, stream=None, pow2=False):
     rows, cols = x.shape
     q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
     s = torch.empty((_cdiv(cols, 128), rows), dtype=torch.float32,
                     device=x.device)
-    fp8bw_quantize_rowwise(x, q, s, stream)
+    fp8bw_quantize_rowwise(x, q, s, stream, pow2=pow2)
     return q, s
 
 
-def quantize_colwise(x, with_rowwise=False, stream=None):
+def quantize_colwise(x, with_rowwise=False, stream=None, pow2=False):
     """-> (q_t, s_t) or (q_t, s_t, q_row, s_row) when with_rowwise."""
     rows, cols = x.shape
     dev = x.device
@@ -178,11 +193,11 @@ def quantize_colwise(x, with_rowwise=False, stream=None):
         q_row = torch.empty((rows, cols), dtype=torch.uint8, device=dev)
         s_row = torch.empty((_cdiv(cols, 128), rows), dtype=torch.float32,
                             device=dev)
-    fp8bw_quantize_colwise(x, q_t, s_t, q_row, s_row, stream)
+    fp8bw_quantize_colwise(x, q_t, s_t, q_row, s_row, stream, pow2=pow2)
     return (q_t, s_t, q_row, s_row) if with_rowwise else (q_t, s_t)
 
 
-def quantize_weight_block(w, transposed=True, stream=None):
+def quantize_weight_block(w, transposed=True, stream=None, pow2=False):
     n, k = w.shape
     dev = w.device
     q = torch.empty((n, k), dtype=torch.uint8, device=dev)
@@ -190,29 +205,31 @@ def quantize_weight_block(w, transposed=True, stream=None):
                     device=dev)
     q_t = torch.empty((k, n), dtype=torch.uint8, device=dev) if transposed \
         else None
-    fp8bw_quantize_weight_block(w, q, s, q_t, stream)
+    fp8bw_quantize_weight_block(w, q, s, q_t, stream, pow2=pow2)
     return q, s, q_t
 
 
-def gemm_fprop(qx, sx, qw, sw, stream=None):
+def gemm_fprop(qx, sx, qw, sw, stream=None, pow2=False):
     y = torch.empty((qx.shape[0], qw.shape[0]), dtype=torch.bfloat16,
                     device=qx.device)
-    fp8bw_gemm_fprop(qx, sx, qw, sw, y, stream)
+    fp8bw_gemm_fprop(qx, sx, qw, sw, y, stream, pow2=pow2)
     return y
 
 
-def gemm_dgrad(qdy, sdy, qw, sw, qw_is_transposed=True, stream=None):
+def gemm_dgrad(qdy, sdy, qw, sw, qw_is_transposed=True, stream=None,
+               pow2=False):
     k = qw.shape[0] if qw_is_transposed else qw.shape[1]
     dx = torch.empty((qdy.shape[0], k), dtype=torch.bfloat16,
                      device=qdy.device)
-    fp8bw_gemm_dgrad(qdy, sdy, qw, qw_is_transposed, sw, dx, stream)
+    fp8bw_gemm_dgrad(qdy, sdy, qw, qw_is_transposed, sw, dx, stream,
+                     pow2=pow2)
     return dx
 
 
-def gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t, stream=None):
+def gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t, stream=None, pow2=False):
     dw = torch.empty((qdy_t.shape[0], qx_t.shape[0]), dtype=torch.bfloat16,
                      device=qdy_t.device)
-    fp8bw_gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t, dw, stream)
+    fp8bw_gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t, dw, stream, pow2=pow2)
     return dw
 
 

@@ -65,7 +65,10 @@ typedef enum fp8bw_status {
     FP8BW_ERR_LAUNCH = -5,         /* the CUDA launch failed */
     FP8BW_ERR_DEVICE_TIMEOUT = -6, /* a bounded device-side wait expired */
     FP8BW_ERR_CUDA = -7,           /* another CUDA runtime/driver call failed */
-    FP8BW_ERR_ALIAS = -8           /* an output overlaps an input */
+    FP8BW_ERR_ALIAS = -8,          /* an output overlaps an input */
+    FP8BW_ERR_SCALE = -9           /* a *_pow2 GEMM read a scale that is not
+                                      a power of two (reported by
+                                      fp8bw_check_device_error) */
 } fp8bw_status;
 
 /* Row-wise 1x128 quantisation of an activation or gradient X[rows, cols]
@@ -158,10 +161,49 @@ int fp8bw_gemm_wgrad_f32(const uint8_t* qdy_t, const float* sdy_t,
                          int64_t n, int64_t k, float* dw, int accumulate,
                          void* stream);
 
+/* ------------------------------------------------------------------------
+ * Power-of-two scales on the tensor cores' block scaling.
+ *
+ * The pages fix blockwise E4M3 with 1x128 activation groups and 128x128
+ * weight blocks, each with one scale (arxiv-wiki summary, "Approach" item
+ * (4)), and say the grouping and scaling follow the DeepSeek-V3 approach
+ * (same page, developer notes, bullet 3); they do not fix the form of the
+ * scale. These entry points use power-of-two scales: s = 2^E with E the
+ * smallest integer such that 448 * 2^E >= amax (E >= -127; an all-zero group
+ * gets s = 1), codes E4M3(x * 2^-E). With such scales the B200 tensor cores
+ * apply the scales themselves (UE8M0 block scaling) and accumulate the whole
+ * contraction in fp32, so the GEMMs need no per-chunk promotion.
+ *
+ * Arguments, layouts, ownership and errors are those of the entry points
+ * without the suffix. Scales stay fp32 (exact powers of two) in the same
+ * layouts; the *_pow2 GEMMs accept only such scales (anything else makes the
+ * next fp8bw_check_device_error return FP8BW_ERR_SCALE, and that output is
+ * undefined). The codes of a *_pow2 quantiser feed only *_pow2 GEMMs.
+ * ------------------------------------------------------------------------ */
+int fp8bw_quantize_rowwise_pow2(const uint16_t* x, int64_t rows, int64_t cols,
+                                uint8_t* q, float* s, void* stream);
+int fp8bw_quantize_colwise_pow2(const uint16_t* x, int64_t rows, int64_t cols,
+                                uint8_t* q_t, float* s_t, uint8_t* q_row,
+                                float* s_row, void* stream);
+int fp8bw_quantize_weight_block_pow2(const uint16_t* w, int64_t n, int64_t k,
+                                     uint8_t* q, float* s, uint8_t* q_t,
+                                     void* stream);
+int fp8bw_gemm_fprop_pow2(const uint8_t* qx, const float* sx,
+                          const uint8_t* qw, const float* sw, int64_t m,
+                          int64_t n, int64_t k, uint16_t* y, void* stream);
+int fp8bw_gemm_dgrad_pow2(const uint8_t* qdy, const float* sdy,
+                          const uint8_t* qw, int qw_is_transposed,
+                          const float* sw, int64_t m, int64_t n, int64_t k,
+                          uint16_t* dx, void* stream);
+int fp8bw_gemm_wgrad_pow2(const uint8_t* qdy_t, const float* sdy_t,
+                          const uint8_t* qx_t, const float* sx_t, int64_t m,
+                          int64_t n, int64_t k, uint16_t* dw, void* stream);
+
 /* Synchronises `stream`, then returns FP8BW_ERR_DEVICE_TIMEOUT if any kernel
  * of this library on the current device recorded an expired wait since the
- * last call (and clears the record), else FP8BW_OK (or FP8BW_ERR_CUDA if the
- * synchronisation itself failed). */
+ * last call, FP8BW_ERR_SCALE if a *_pow2 GEMM recorded a scale that is not a
+ * power of two (and clears the record), else FP8BW_OK (or FP8BW_ERR_CUDA if
+ * the synchronisation itself failed). */
 int fp8bw_check_device_error(void* stream);
 
 /* Static, NUL-terminated description of a status code. */

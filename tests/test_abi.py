@@ -15,6 +15,7 @@ HEADER = os.path.join(ROOT, "include", "fp8bw.h")
 
 OK, E_NULL, E_SHAPE, E_ALIGN, E_DEVICE, E_LAUNCH, E_TIMEOUT, E_CUDA, E_ALIAS = \
     0, -1, -2, -3, -4, -5, -6, -7, -8
+E_SCALE = -9
 
 A = 0x10000000   # fake, 16-byte aligned, never dereferenced
 B = 0x20000000
@@ -36,16 +37,16 @@ def lib():
 
 def test_every_declared_symbol_is_exported(lib):
     names = declared_functions()
-    assert len(names) == 10
+    assert len(names) == 16
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(_native.SIGNATURES)
 
 
 def test_status_strings_and_version(lib):
-    assert lib.fp8bw_version() == 101
+    assert lib.fp8bw_version() == 102
     for st in (OK, E_NULL, E_SHAPE, E_ALIGN, E_DEVICE, E_LAUNCH, E_TIMEOUT,
-               E_CUDA, E_ALIAS):
+               E_CUDA, E_ALIAS, E_SCALE):
         s = lib.fp8bw_status_string(st).decode()
         assert s and s != "unknown status"
     assert lib.fp8bw_status_string(12345).decode() == "unknown status"
@@ -68,6 +69,11 @@ def test_null_pointers_rejected(lib):
                                 None) == E_NULL
     assert lib.fp8bw_gemm_wgrad_f32(A, B, C, D, 128, 128, 128, None, 1,
                                     None) == E_NULL
+    assert lib.fp8bw_quantize_rowwise_pow2(None, 128, 128, B, C, None) == E_NULL
+    assert lib.fp8bw_gemm_fprop_pow2(A, B, C, None, 128, 128, 128, E,
+                                     None) == E_NULL
+    assert lib.fp8bw_gemm_wgrad_pow2(A, B, C, D, 128, 128, 128, None,
+                                     None) == E_NULL
 
 
 @pytest.mark.parametrize("rows,cols", [(-16, 128), (128, -16), (100, 128),
@@ -86,6 +92,10 @@ def test_bad_shapes_rejected(lib, rows, cols):
                                 None) == E_SHAPE
     assert lib.fp8bw_gemm_wgrad_f32(A, B, C, D, cols, 128, rows, E, 0,
                                     None) == E_SHAPE
+    assert lib.fp8bw_quantize_colwise_pow2(A, rows, cols, B, C, None, None,
+                                           None) == E_SHAPE
+    assert lib.fp8bw_gemm_dgrad_pow2(A, B, C, 1, D, 128, rows, cols, E,
+                                     None) == E_SHAPE
 
 
 def test_misaligned_pointers_rejected(lib):
@@ -102,6 +112,8 @@ def test_misaligned_pointers_rejected(lib):
                                 None) == E_ALIGN
     assert lib.fp8bw_gemm_wgrad_f32(A, B, C, D, 128, 128, 128, E + 8, 1,
                                     None) == E_ALIGN
+    assert lib.fp8bw_quantize_weight_block_pow2(A, 128, 128, B, C, D + 8,
+                                                None) == E_ALIGN
 
 
 def test_aliased_outputs_rejected(lib):
