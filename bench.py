@@ -349,6 +349,61 @@ def time_next_rows(o, bufs, stream, warmup, rounds):
         "what": "dW (fp32) += dY^T X for the QKV, O, gate/up and down "
                 "linears at M=%d, in turn; timed after the step" % TOKENS}}
 
+    # fprop and dgrad that also quantise their own bf16 output row-wise,
+    # against the same GEMMs followed by the row-wise quantiser.
+    def seq_time(seq, rounds=3):
+        with torch.cuda.stream(stream):
+            for _ in range(warmup):
+                for fn in seq:
+                    fn()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b_ = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            a.record(stream)
+            for _ in range(rounds):
+                for fn in seq:
+                    fn()
+            b_.record(stream)
+        torch.cuda.synchronize()
+        o.fp8bw_check_device_error(stream)
+        return a.elapsed_time(b_) / rounds
+
+    fused, unfused = [], []
+    for b in bufs:
+        m = TOKENS
+        u8, f32 = torch.uint8, torch.float32
+        qy = torch.empty((m, b.n), dtype=u8, device=dev)
+        sy = torch.empty(((b.n + 127) // 128, m), dtype=f32, device=dev)
+        qdx = torch.empty((m, b.k), dtype=u8, device=dev)
+        sdx = torch.empty(((b.k + 127) // 128, m), dtype=f32, device=dev)
+        fused += [
+            (lambda b=b, qy=qy, sy=sy: o.fp8bw_gemm_fprop_quant(
+                b.qx, b.sx, b.qw, b.sw, b.y, qy, sy, stream)),
+            (lambda b=b, qdx=qdx, sdx=sdx: o.fp8bw_gemm_dgrad_quant(
+                b.qdy, b.sdy, b.qw_t, 1, b.sw, b.dx, qdx, sdx, stream))]
+        unfused += [
+            (lambda b=b: o.fp8bw_gemm_fprop(b.qx, b.sx, b.qw, b.sw, b.y,
+                                            stream)),
+            (lambda b=b, qy=qy, sy=sy: o.fp8bw_quantize_rowwise(b.y, qy, sy,
+                                                                stream)),
+            (lambda b=b: o.fp8bw_gemm_dgrad(b.qdy, b.sdy, b.qw_t, 1, b.sw,
+                                            b.dx, stream)),
+            (lambda b=b, qdx=qdx, sdx=sdx: o.fp8bw_quantize_rowwise(
+                b.dx, qdx, sdx, stream))]
+    t_f = seq_time(fused)
+    t_u = seq_time(unfused)
+    gfl = 2 * sum(2 * TOKENS * b.n * b.k for b in bufs)
+    out["gemm_fused_rowwise_quant"] = {
+        "achieved": gfl / (t_f * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "ms_fused": t_f, "ms_gemm_then_quantiser": t_u,
+        "saved_frac": 1.0 - t_f / t_u,
+        "what": "fprop and dgrad of the four linears (M=%d) writing bf16 "
+                "plus the row-wise E4M3 codes and scales of that output, "
+                "against the same GEMMs followed by the row-wise quantiser; "
+                "timed after the step" % TOKENS}
+    del qy, sy, qdx, sdx
+
     # The whole step again with power-of-two scales (quantisers and GEMMs on
     # the tensor cores' UE8M0 block scaling), same buffers and order.
     step = []

@@ -173,6 +173,8 @@ struct GemmProblem {
   void* out;         // [mo][no]: bf16 (kOutBf16) or fp32
   int out_mode;      // gemm::kOutBf16 / kOutF32 / kOutF32Add
   bool pow2;         // power-of-two scales on the hardware block-scaled MMA
+  uint8_t* q_out;    // kOutBf16Q: row-wise codes of the bf16 output [mo][no]
+  float* s_out;      // kOutBf16Q: their scales [ceil(no/128)][mo]
 };
 
 // CTA-pair kernel: 256 x 256 output tiles on clusters of two CTAs.
@@ -225,7 +227,7 @@ int launch_gemm_pair(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t s
     st = encode_u8_2d(&tm_b, p.b, static_cast<uint64_t>(p.kc), static_cast<uint64_t>(p.no),
                       BN / 2);
   if (st != FP8BW_OK) return st;
-  if (OUT == gemm::kOutBf16)
+  if (gemm::out_is_bf16(OUT))
     st = encode_bf16_out(&tm_out, p.out, static_cast<uint64_t>(p.no),
                          static_cast<uint64_t>(p.mo));
   else
@@ -245,6 +247,8 @@ int launch_gemm_pair(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t s
   g.sbc = p.sbc;
   g.nblk = static_cast<int>(cdiv(p.no, 128));
   g.out = p.out;
+  g.q_out = p.q_out;
+  g.s_out = p.s_out;
   const int64_t tiles = static_cast<int64_t>(g.tiles_m) * g.tiles_n;
   const int clusters = static_cast<int>(std::min<int64_t>(tiles, max_clusters));
   kernel<<<2 * clusters, gemm::kThreads, L::kAlloc, stream>>>(tm_a, tm_b, tm_out, g);
@@ -321,11 +325,14 @@ int run_gemm(const GemmProblem& p, cudaStream_t stream) {
   if (p.kc == 0) {
     // An empty contraction: the product is zero (adding it changes nothing).
     if (p.out_mode == gemm::kOutF32Add) return FP8BW_OK;
-    const size_t esize = p.out_mode == gemm::kOutBf16 ? 2 : 4;
-    return cudaMemsetAsync(p.out, 0, static_cast<size_t>(p.mo * p.no) * esize, stream) ==
-                   cudaSuccess
-               ? FP8BW_OK
-               : FP8BW_ERR_CUDA;
+    const size_t esize = gemm::out_is_bf16(p.out_mode) ? 2 : 4;
+    if (cudaMemsetAsync(p.out, 0, static_cast<size_t>(p.mo * p.no) * esize, stream) !=
+        cudaSuccess)
+      return FP8BW_ERR_CUDA;
+    if (p.out_mode != gemm::kOutBf16Q) return FP8BW_OK;
+    // ... and its row-wise quantisation is that of a zero matrix
+    return launch_quantize(kModeRow, false, static_cast<const uint16_t*>(p.out), p.mo, p.no,
+                           p.q_out, p.s_out, nullptr, nullptr, nullptr, dev.sm_count, stream);
   }
   if (cdiv(p.mo, 256) * cdiv(p.no, 256) > (int64_t(1) << 30)) return FP8BW_ERR_SHAPE;
   if (p.pow2) {
@@ -338,6 +345,10 @@ int run_gemm(const GemmProblem& p, cudaStream_t stream) {
     return launch_gemm_pair<GEMM_BN_VEC, true, false, gemm::kOutF32>(p, dev, stream);
   if (p.vec_b && p.out_mode == gemm::kOutF32Add)
     return launch_gemm_pair<GEMM_BN_VEC, true, false, gemm::kOutF32Add>(p, dev, stream);
+  if (p.out_mode == gemm::kOutBf16Q && !p.vec_b) {
+    if (p.b_mn) return launch_gemm_pair<256, false, true, gemm::kOutBf16Q>(p, dev, stream);
+    return launch_gemm_pair<256, false, false, gemm::kOutBf16Q>(p, dev, stream);
+  }
   if (p.out_mode != gemm::kOutBf16) return FP8BW_ERR_LAUNCH;
   if (p.vec_b) return launch_gemm_pair<GEMM_BN_VEC, true, false>(p, dev, stream);
   if (p.b_mn) return launch_gemm_pair<256, false, true>(p, dev, stream);
@@ -351,7 +362,7 @@ using namespace fp8bw;
 
 extern "C" {
 
-int fp8bw_version(void) { return 102; }
+int fp8bw_version(void) { return 103; }
 
 const char* fp8bw_status_string(int status) {
   switch (status) {
@@ -471,18 +482,34 @@ int fp8bw_quantize_weight_block_pow2(const uint16_t* w, int64_t n, int64_t k, ui
 
 namespace {
 
+// Output checks of a GEMM with a bf16 output out[rows, cols] and, optionally,
+// its row-wise quantisation (q [rows, cols], s [ceil(cols/128)][rows]):
+// alignment, and no overlap with the inputs or with each other.
+int quant_outputs_status(const void* out, int64_t rows, int64_t cols, const uint8_t* q,
+                         const float* s, const Range* ins, int nins) {
+  if (!aligned16(q) || !aligned16(s)) return FP8BW_ERR_ALIGN;
+  const Range ro = range_of(out, rows * cols * 2);
+  const Range rq = range_of(q, q ? rows * cols : 0);
+  const Range rs = range_of(s, s ? cdiv(cols, 128) * rows * 4 : 0);
+  for (int i = 0; i < nins; ++i)
+    if (overlap(ro, ins[i]) || overlap(rq, ins[i]) || overlap(rs, ins[i])) return FP8BW_ERR_ALIAS;
+  if (overlap(ro, rq) || overlap(ro, rs) || overlap(rq, rs)) return FP8BW_ERR_ALIAS;
+  return FP8BW_OK;
+}
+
 int gemm_fprop(bool pow2, const uint8_t* qx, const float* sx, const uint8_t* qw, const float* sw,
-               int64_t m, int64_t n, int64_t k, uint16_t* y, void* stream) {
+               int64_t m, int64_t n, int64_t k, uint16_t* y, uint8_t* qy, float* sy,
+               void* stream) {
   if (!dim_ok(m) || !dim_ok(n) || !dim_ok(k)) return FP8BW_ERR_SHAPE;
   if (missing(qx, m * k) || missing(sx, cdiv(k, 128) * m) || missing(qw, n * k) ||
       missing(sw, cdiv(n, 128) * cdiv(k, 128)) || missing(y, m * n))
     return FP8BW_ERR_NULL;
   if (!aligned16(qx) || !aligned16(sx) || !aligned16(qw) || !aligned16(sw) || !aligned16(y))
     return FP8BW_ERR_ALIGN;
-  const Range ry = range_of(y, m * n * 2);
-  if (overlap(ry, range_of(qx, m * k)) || overlap(ry, range_of(sx, cdiv(k, 128) * m * 4)) ||
-      overlap(ry, range_of(qw, n * k)) || overlap(ry, range_of(sw, cdiv(n, 128) * cdiv(k, 128) * 4)))
-    return FP8BW_ERR_ALIAS;
+  const Range ins[4] = {range_of(qx, m * k), range_of(sx, cdiv(k, 128) * m * 4),
+                        range_of(qw, n * k), range_of(sw, cdiv(n, 128) * cdiv(k, 128) * 4)};
+  const int ost = quant_outputs_status(y, m, n, qy, sy, ins, 4);
+  if (ost != FP8BW_OK) return ost;
   GemmProblem p{};
   p.a = qx;
   p.b = qw;
@@ -497,22 +524,25 @@ int gemm_fprop(bool pow2, const uint8_t* qx, const float* sx, const uint8_t* qw,
   p.sbc = 1;
   p.out = y;
   p.pow2 = pow2;
+  p.q_out = qy;
+  p.s_out = sy;
+  p.out_mode = qy ? gemm::kOutBf16Q : gemm::kOutBf16;
   return run_gemm(p, static_cast<cudaStream_t>(stream));
 }
 
 int gemm_dgrad(bool pow2, const uint8_t* qdy, const float* sdy, const uint8_t* qw,
                int qw_is_transposed, const float* sw, int64_t m, int64_t n, int64_t k,
-               uint16_t* dx, void* stream) {
+               uint16_t* dx, uint8_t* qdx, float* sdx, void* stream) {
   if (!dim_ok(m) || !dim_ok(n) || !dim_ok(k)) return FP8BW_ERR_SHAPE;
   if (missing(qdy, m * n) || missing(sdy, cdiv(n, 128) * m) || missing(qw, n * k) ||
       missing(sw, cdiv(n, 128) * cdiv(k, 128)) || missing(dx, m * k))
     return FP8BW_ERR_NULL;
   if (!aligned16(qdy) || !aligned16(sdy) || !aligned16(qw) || !aligned16(sw) || !aligned16(dx))
     return FP8BW_ERR_ALIGN;
-  const Range rd = range_of(dx, m * k * 2);
-  if (overlap(rd, range_of(qdy, m * n)) || overlap(rd, range_of(sdy, cdiv(n, 128) * m * 4)) ||
-      overlap(rd, range_of(qw, n * k)) || overlap(rd, range_of(sw, cdiv(n, 128) * cdiv(k, 128) * 4)))
-    return FP8BW_ERR_ALIAS;
+  const Range ins[4] = {range_of(qdy, m * n), range_of(sdy, cdiv(n, 128) * m * 4),
+                        range_of(qw, n * k), range_of(sw, cdiv(n, 128) * cdiv(k, 128) * 4)};
+  const int ost = quant_outputs_status(dx, m, k, qdx, sdx, ins, 4);
+  if (ost != FP8BW_OK) return ost;
   GemmProblem p{};
   p.a = qdy;
   p.b = qw;
@@ -527,6 +557,9 @@ int gemm_dgrad(bool pow2, const uint8_t* qdy, const float* sdy, const uint8_t* q
   p.sbc = cdiv(k, 128);
   p.out = dx;
   p.pow2 = pow2;
+  p.q_out = qdx;
+  p.s_out = sdx;
+  p.out_mode = qdx ? gemm::kOutBf16Q : gemm::kOutBf16;
   return run_gemm(p, static_cast<cudaStream_t>(stream));
 }
 
@@ -536,24 +569,42 @@ extern "C" {
 
 int fp8bw_gemm_fprop(const uint8_t* qx, const float* sx, const uint8_t* qw, const float* sw,
                      int64_t m, int64_t n, int64_t k, uint16_t* y, void* stream) {
-  return gemm_fprop(false, qx, sx, qw, sw, m, n, k, y, stream);
+  return gemm_fprop(false, qx, sx, qw, sw, m, n, k, y, nullptr, nullptr, stream);
 }
 
 int fp8bw_gemm_dgrad(const uint8_t* qdy, const float* sdy, const uint8_t* qw,
                      int qw_is_transposed, const float* sw, int64_t m, int64_t n, int64_t k,
                      uint16_t* dx, void* stream) {
-  return gemm_dgrad(false, qdy, sdy, qw, qw_is_transposed, sw, m, n, k, dx, stream);
+  return gemm_dgrad(false, qdy, sdy, qw, qw_is_transposed, sw, m, n, k, dx, nullptr, nullptr,
+                    stream);
+}
+
+int fp8bw_gemm_fprop_quant(const uint8_t* qx, const float* sx, const uint8_t* qw,
+                           const float* sw, int64_t m, int64_t n, int64_t k, uint16_t* y,
+                           uint8_t* qy, float* sy, void* stream) {
+  if (missing(qy, m * n) || missing(sy, cdiv(n, 128) * m)) return FP8BW_ERR_NULL;
+  if (m * n > 0 && (qy == nullptr || sy == nullptr)) return FP8BW_ERR_NULL;
+  return gemm_fprop(false, qx, sx, qw, sw, m, n, k, y, qy, sy, stream);
+}
+
+int fp8bw_gemm_dgrad_quant(const uint8_t* qdy, const float* sdy, const uint8_t* qw,
+                           int qw_is_transposed, const float* sw, int64_t m, int64_t n,
+                           int64_t k, uint16_t* dx, uint8_t* qdx, float* sdx, void* stream) {
+  if (missing(qdx, m * k) || missing(sdx, cdiv(k, 128) * m)) return FP8BW_ERR_NULL;
+  if (m * k > 0 && (qdx == nullptr || sdx == nullptr)) return FP8BW_ERR_NULL;
+  return gemm_dgrad(false, qdy, sdy, qw, qw_is_transposed, sw, m, n, k, dx, qdx, sdx, stream);
 }
 
 int fp8bw_gemm_fprop_pow2(const uint8_t* qx, const float* sx, const uint8_t* qw, const float* sw,
                           int64_t m, int64_t n, int64_t k, uint16_t* y, void* stream) {
-  return gemm_fprop(true, qx, sx, qw, sw, m, n, k, y, stream);
+  return gemm_fprop(true, qx, sx, qw, sw, m, n, k, y, nullptr, nullptr, stream);
 }
 
 int fp8bw_gemm_dgrad_pow2(const uint8_t* qdy, const float* sdy, const uint8_t* qw,
                           int qw_is_transposed, const float* sw, int64_t m, int64_t n,
                           int64_t k, uint16_t* dx, void* stream) {
-  return gemm_dgrad(true, qdy, sdy, qw, qw_is_transposed, sw, m, n, k, dx, stream);
+  return gemm_dgrad(true, qdy, sdy, qw, qw_is_transposed, sw, m, n, k, dx, nullptr, nullptr,
+                    stream);
 }
 
 }  // extern "C"
@@ -570,7 +621,7 @@ int wgrad_common(const uint8_t* qdy_t, const float* sdy_t, const uint8_t* qx_t,
   if (!aligned16(qdy_t) || !aligned16(sdy_t) || !aligned16(qx_t) || !aligned16(sx_t) ||
       !aligned16(dw))
     return FP8BW_ERR_ALIGN;
-  const int64_t esize = out_mode == gemm::kOutBf16 ? 2 : 4;
+  const int64_t esize = gemm::out_is_bf16(out_mode) ? 2 : 4;
   const Range rd = range_of(dw, n * k * esize);
   if (overlap(rd, range_of(qdy_t, n * m)) || overlap(rd, range_of(sdy_t, cdiv(m, 128) * n * 4)) ||
       overlap(rd, range_of(qx_t, k * m)) || overlap(rd, range_of(sx_t, cdiv(m, 128) * k * 4)))

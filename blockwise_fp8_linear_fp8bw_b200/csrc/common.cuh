@@ -4,6 +4,8 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include "../../include/fp8bw.h"
@@ -466,6 +468,90 @@ __host__ __device__ constexpr uint32_t idesc_e4m3(int m, int n, bool b_mn_major)
   return (1u << 4) | ((b_mn_major ? 1u : 0u) << 16) |
          (static_cast<uint32_t>(n >> 3) << 17) |
          (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+// ---------------------------------------------------------------------------
+// E4M3 group quantisation, shared by the quantisers and the GEMM epilogue
+// that quantises its own output (same arithmetic, bit for bit).
+// Reading of the scale (not printed on the pages): qscale = 448/amax,
+// s = amax/448 (fp32, round-to-nearest-even), amax == 0 or an overflowing
+// qscale gives qscale = s = 1; code = E4M3_satfinite_rn(x * qscale).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float bf16_lo(uint32_t w) {
+  return __uint_as_float(w << 16);
+}
+__device__ __forceinline__ float bf16_hi(uint32_t w) {
+  return __uint_as_float(w & 0xFFFF0000u);
+}
+
+// qscale / s pair of a group (see the file comment).
+__device__ __forceinline__ void group_scale(float amax, float& qscale,
+                                            float& s) {
+  float q = __fdiv_rn(448.0f, amax);
+  if (amax == 0.0f || !isfinite(q)) {
+    qscale = 1.0f;
+    s = 1.0f;
+  } else {
+    qscale = q;
+    s = __fdiv_rn(amax, 448.0f);
+  }
+}
+
+// Power-of-two form: s = 2^E with E the smallest integer such that
+// 448 * 2^E >= amax, clamped below at -127 (a finite bf16 amax <= 3.39e38
+// keeps E <= 120, so qscale = 2^-E is always a normal float). With
+// amax = (1 + f) * 2^(ef - 127): E = ef - 135 when 1 + f <= 1.75 (448 =
+// 1.75 * 2^8), else ef - 134; a subnormal amax gives E = -127. All integer
+// work on the bits, so the result is exact.
+__device__ __forceinline__ void group_scale_pow2(float amax, float& qscale, float& s) {
+  if (amax == 0.0f || !isfinite(amax)) {
+    qscale = 1.0f;
+    s = 1.0f;
+    return;
+  }
+  const uint32_t b = __float_as_uint(amax);
+  const int ef = static_cast<int>(b >> 23);
+  int e = ef == 0 ? -127 : ef - 135 + ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+  e = max(-127, min(120, e));
+  s = e >= -126 ? __uint_as_float(static_cast<uint32_t>(e + 127) << 23)
+                : __uint_as_float(0x00400000u);   // 2^-127, a subnormal
+  qscale = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+}
+
+template <bool POW2>
+__device__ __forceinline__ void scale_of(float amax, float& qscale, float& s) {
+  if constexpr (POW2)
+    group_scale_pow2(amax, qscale, s);
+  else
+    group_scale(amax, qscale, s);
+}
+
+// |x| of two packed bf16 values (clears both sign bits; exact).
+__device__ __forceinline__ uint32_t abs_bf16x2(uint32_t w) { return w & 0x7FFF7FFFu; }
+
+// Element-wise max of two packed non-negative bf16 pairs (exact).
+__device__ __forceinline__ uint32_t max_bf16x2(uint32_t a, uint32_t b) {
+  __nv_bfloat162 r = __hmax2(*reinterpret_cast<__nv_bfloat162*>(&a),
+                             *reinterpret_cast<__nv_bfloat162*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// The larger of the two bf16 halves, as fp32 (exact).
+__device__ __forceinline__ float max_halves(uint32_t w) {
+  return fmaxf(bf16_lo(w), bf16_hi(w));
+}
+
+// Two fp32 values -> two E4M3 codes (round to nearest even, satfinite);
+// `a` lands in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
+  return static_cast<uint32_t>(
+      __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
+}
+
+// x * qscale for the two bf16 values of a packed pair, one IEEE fp32
+// multiply each (round to nearest even), as one f32x2 instruction.
+__device__ __forceinline__ void scale_pair(uint32_t w, float qs, float& t0, float& t1) {
+  fmul2(t0, t1, bf16_lo(w), bf16_hi(w), qs, qs);
 }
 
 // ---------------------------------------------------------------------------

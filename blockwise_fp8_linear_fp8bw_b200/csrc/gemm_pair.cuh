@@ -83,6 +83,13 @@ static_assert(4 * 32 * kProducerRegs + kNumEpiWarps * 32 * kEpilogueRegs ==
 constexpr int kOutBf16 = 0;       // bf16 store
 constexpr int kOutF32 = 1;        // fp32 store
 constexpr int kOutF32Add = 2;     // fp32 add into the existing output (TMA reduce-add)
+constexpr int kOutBf16Q = 3;      // bf16 store + row-wise E4M3 quantisation of that bf16
+                                  // output (block-scale mode only)
+
+// Element type of the output tensor (the TMA map and the staging boxes).
+__host__ __device__ constexpr bool out_is_bf16(int out) {
+  return out == kOutBf16 || out == kOutBf16Q;
+}
 
 struct Args {
   int mo, no, kc;             // output rows, output columns, contraction length
@@ -92,6 +99,8 @@ struct Args {
   int64_t sbj, sbc;
   int nblk;                   // number of 128-wide output column blocks
   void* out;                  // [mo][no], bf16 or fp32 (written through tm_out)
+  uint8_t* q_out;             // kOutBf16Q: codes [mo][no]
+  float* s_out;               // kOutBf16Q: scales [ceil(no/128)][mo]
 };
 
 __device__ __forceinline__ void setmaxnreg_dec() {
@@ -142,6 +151,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   constexpr int kPairStages = L::kStages;
   constexpr int kBufs = L::kTmemBufs;
   static_assert(!B_MN || BN == 256, "MN-major B uses full 128-element swizzle atoms");
+  static_assert(OUT != kOutBf16Q || (!VEC_B && BN == 256),
+                "the fused quantisation needs one 128-column group per thread");
   constexpr int kHalf = BN / 2;                      // columns per epilogue thread
   constexpr uint32_t kIdesc = idesc_e4m3(2 * BM, BN, B_MN);
 
@@ -463,9 +474,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
       const int y0 = tm * (2 * BM) + static_cast<int>(rank) * BM + q * 32;
       const int x0 = tn * BN + h * kHalf;
+      // kOutBf16Q: this thread's 128 columns of its row are exactly one 1x128
+      // group (x0 is a multiple of 128) of the bf16 output; quantise the bf16
+      // values as the row-wise quantiser would.
+      float qscale = 1.0f;
+      if constexpr (OUT == kOutBf16Q) {
+        uint32_t mx = 0u;
+#pragma unroll
+        for (int j = 0; j < kHalf / 2; ++j)
+          mx = max_bf16x2(mx, abs_bf16x2(pack_bf16x2(acc[2 * j], acc[2 * j + 1])));
+        float sc;
+        group_scale(max_halves(mx), qscale, sc);
+        const int grow = y0 + lane;
+        if (grow < g.mo && x0 < g.no) g.s_out[static_cast<int64_t>(x0 / 128) * g.mo + grow] = sc;
+      }
       // One 2 KB staging box per warp: 32 rows of 64 bytes (32 bf16 or 16
       // fp32 columns), 64-byte swizzle (16-byte unit j of row r at j ^ (r/2 % 4)).
-      constexpr int kBoxCols = OUT == kOutBf16 ? 32 : 16;
+      constexpr int kBoxCols = out_is_bf16(OUT) ? 32 : 16;
 #pragma unroll
       for (int gi = 0; gi < kHalf / kBoxCols; ++gi) {
         if (x0 + gi * kBoxCols >= g.no || y0 >= g.mo) continue;
@@ -502,26 +527,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
           }
         } else {
+          uint32_t codes[8];   // kOutBf16Q: this row's 32 codes of the box
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             uint32_t w0, w1, w2, w3;
-          if constexpr (OUT == kOutBf16) {
-            const float* v = acc + gi * 32 + j * 8;
-            w0 = pack_bf16x2(v[0], v[1]);
-            w1 = pack_bf16x2(v[2], v[3]);
-            w2 = pack_bf16x2(v[4], v[5]);
-            w3 = pack_bf16x2(v[6], v[7]);
-          } else {
-            const float* v = acc + gi * 16 + j * 4;
-            w0 = __float_as_uint(v[0]);
-            w1 = __float_as_uint(v[1]);
-            w2 = __float_as_uint(v[2]);
-            w3 = __float_as_uint(v[3]);
-          }
+            if constexpr (out_is_bf16(OUT)) {
+              const float* v = acc + gi * 32 + j * 8;
+              w0 = pack_bf16x2(v[0], v[1]);
+              w1 = pack_bf16x2(v[2], v[3]);
+              w2 = pack_bf16x2(v[4], v[5]);
+              w3 = pack_bf16x2(v[6], v[7]);
+              if constexpr (OUT == kOutBf16Q) {
+                float t[8];
+                scale_pair(w0, qscale, t[0], t[1]);
+                scale_pair(w1, qscale, t[2], t[3]);
+                scale_pair(w2, qscale, t[4], t[5]);
+                scale_pair(w3, qscale, t[6], t[7]);
+                codes[2 * j] = e4m3x2(t[0], t[1]) | (e4m3x2(t[2], t[3]) << 16);
+                codes[2 * j + 1] = e4m3x2(t[4], t[5]) | (e4m3x2(t[6], t[7]) << 16);
+              }
+            } else {
+              const float* v = acc + gi * 16 + j * 4;
+              w0 = __float_as_uint(v[0]);
+              w1 = __float_as_uint(v[1]);
+              w2 = __float_as_uint(v[2]);
+              w3 = __float_as_uint(v[3]);
+            }
             const uint32_t dst = stage_out + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4);
             asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(w0),
                          "r"(w1), "r"(w2), "r"(w3)
                          : "memory");
+          }
+          if constexpr (OUT == kOutBf16Q) {
+            const int grow = y0 + lane;
+            if (grow < g.mo) {
+              uint8_t* dst = g.q_out + static_cast<int64_t>(grow) * g.no + x0 + gi * 32;
+              *reinterpret_cast<uint4*>(dst) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+              if (x0 + gi * 32 + 16 < g.no)
+                *reinterpret_cast<uint4*>(dst + 16) =
+                    make_uint4(codes[4], codes[5], codes[6], codes[7]);
+            }
           }
         }
         fence_proxy_async_smem();

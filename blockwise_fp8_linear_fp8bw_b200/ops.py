@@ -165,6 +165,38 @@ def fp8bw_gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, dw, accumulate=False,
            "fp8bw_gemm_wgrad_f32")
 
 
+def fp8bw_gemm_fprop_quant(qx, sx, qw, sw, y, qy, sy, stream=None):
+    m, k = qx.shape
+    n = qw.shape[0]
+    _expect(qw, torch.uint8, (n, k), "qw")
+    _expect(sx, torch.float32, (_cdiv(k, 128), m), "sx")
+    _expect(sw, torch.float32, (_cdiv(n, 128), _cdiv(k, 128)), "sw")
+    _expect(y, torch.bfloat16, (m, n), "y")
+    _expect(qy, torch.uint8, (m, n), "qy")
+    _expect(sy, torch.float32, (_cdiv(n, 128), m), "sy")
+    _check(_lib.fp8bw_gemm_fprop_quant(_ptr(qx), _ptr(sx), _ptr(qw), _ptr(sw),
+                                       m, n, k, _ptr(y), _ptr(qy), _ptr(sy),
+                                       _stream(stream)),
+           "fp8bw_gemm_fprop_quant")
+
+
+def fp8bw_gemm_dgrad_quant(qdy, sdy, qw, qw_is_transposed, sw, dx, qdx, sdx,
+                           stream=None):
+    m, n = qdy.shape
+    k = qw.shape[0] if qw_is_transposed else qw.shape[1]
+    _expect(qw, torch.uint8, (k, n) if qw_is_transposed else (n, k), "qw")
+    _expect(sdy, torch.float32, (_cdiv(n, 128), m), "sdy")
+    _expect(sw, torch.float32, (_cdiv(n, 128), _cdiv(k, 128)), "sw")
+    _expect(dx, torch.bfloat16, (m, k), "dx")
+    _expect(qdx, torch.uint8, (m, k), "qdx")
+    _expect(sdx, torch.float32, (_cdiv(k, 128), m), "sdx")
+    _check(_lib.fp8bw_gemm_dgrad_quant(_ptr(qdy), _ptr(sdy), _ptr(qw),
+                                       1 if qw_is_transposed else 0, _ptr(sw),
+                                       m, n, k, _ptr(dx), _ptr(qdx), _ptr(sdx),
+                                       _stream(stream)),
+           "fp8bw_gemm_dgrad_quant")
+
+
 def fp8bw_check_device_error(stream=None):
     _check(_lib.fp8bw_check_device_error(_stream(stream)),
            "fp8bw_check_device_error")
@@ -243,3 +275,27 @@ def gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, main_grad=None, stream=None):
                      device=qdy_t.device)
     fp8bw_gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, dw, False, stream)
     return dw
+
+
+def gemm_fprop_quant(qx, sx, qw, sw, stream=None):
+    """-> (y, qy, sy): the bf16 product and its row-wise quantisation."""
+    m, n = qx.shape[0], qw.shape[0]
+    dev = qx.device
+    y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+    qy = torch.empty((m, n), dtype=torch.uint8, device=dev)
+    sy = torch.empty((_cdiv(n, 128), m), dtype=torch.float32, device=dev)
+    fp8bw_gemm_fprop_quant(qx, sx, qw, sw, y, qy, sy, stream)
+    return y, qy, sy
+
+
+def gemm_dgrad_quant(qdy, sdy, qw, sw, qw_is_transposed=True, stream=None):
+    """-> (dx, qdx, sdx): the bf16 product and its row-wise quantisation."""
+    m = qdy.shape[0]
+    k = qw.shape[0] if qw_is_transposed else qw.shape[1]
+    dev = qdy.device
+    dx = torch.empty((m, k), dtype=torch.bfloat16, device=dev)
+    qdx = torch.empty((m, k), dtype=torch.uint8, device=dev)
+    sdx = torch.empty((_cdiv(k, 128), m), dtype=torch.float32, device=dev)
+    fp8bw_gemm_dgrad_quant(qdy, sdy, qw, qw_is_transposed, sw, dx, qdx, sdx,
+                           stream)
+    return dx, qdx, sdx

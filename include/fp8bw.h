@@ -161,6 +161,28 @@ int fp8bw_gemm_wgrad_f32(const uint8_t* qdy_t, const float* sdy_t,
                          int64_t n, int64_t k, float* dw, int accumulate,
                          void* stream);
 
+/* fprop / dgrad that also quantise their own bf16 output row-wise, for a
+ * linear that consumes it next: the same y (dx) as fp8bw_gemm_fprop
+ * (fp8bw_gemm_dgrad), plus exactly what fp8bw_quantize_rowwise would write
+ * for that bf16 output, without reading it back from memory.
+ *   qy, sy   : E4M3 codes [m, n] and scales [ceil(n/128)][m] of y (out)
+ *   qdx, sdx : E4M3 codes [m, k] and scales [ceil(k/128)][m] of dx (out)
+ * Other arguments and errors as the calls without the suffix; the extra
+ * outputs are required (non-NULL when non-empty), 16-byte aligned and must
+ * not overlap any input or each other.
+ * Source: paperlayer.ai summary, Appendix C, "FP8 implementation pipeline"
+ * (bf16 hidden flow between E4M3 GEMMs; the 1x128 row groups of the
+ * arxiv-wiki summary, Approach item (4)). */
+int fp8bw_gemm_fprop_quant(const uint8_t* qx, const float* sx,
+                           const uint8_t* qw, const float* sw, int64_t m,
+                           int64_t n, int64_t k, uint16_t* y, uint8_t* qy,
+                           float* sy, void* stream);
+int fp8bw_gemm_dgrad_quant(const uint8_t* qdy, const float* sdy,
+                           const uint8_t* qw, int qw_is_transposed,
+                           const float* sw, int64_t m, int64_t n, int64_t k,
+                           uint16_t* dx, uint8_t* qdx, float* sdx,
+                           void* stream);
+
 /* ------------------------------------------------------------------------
  * Power-of-two scales on the tensor cores' block scaling.
  *

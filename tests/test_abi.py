@@ -37,14 +37,14 @@ def lib():
 
 def test_every_declared_symbol_is_exported(lib):
     names = declared_functions()
-    assert len(names) == 16
+    assert len(names) == 18
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(_native.SIGNATURES)
 
 
 def test_status_strings_and_version(lib):
-    assert lib.fp8bw_version() == 102
+    assert lib.fp8bw_version() == 103
     for st in (OK, E_NULL, E_SHAPE, E_ALIGN, E_DEVICE, E_LAUNCH, E_TIMEOUT,
                E_CUDA, E_ALIAS, E_SCALE):
         s = lib.fp8bw_status_string(st).decode()
@@ -74,6 +74,11 @@ def test_null_pointers_rejected(lib):
                                      None) == E_NULL
     assert lib.fp8bw_gemm_wgrad_pow2(A, B, C, D, 128, 128, 128, None,
                                      None) == E_NULL
+    # the fused quantisation outputs are required
+    assert lib.fp8bw_gemm_fprop_quant(A, B, C, D, 128, 128, 128, E, None,
+                                      E + 0x100000, None) == E_NULL
+    assert lib.fp8bw_gemm_dgrad_quant(A, B, C, 1, D, 128, 128, 128, E,
+                                      E + 0x100000, None, None) == E_NULL
 
 
 @pytest.mark.parametrize("rows,cols", [(-16, 128), (128, -16), (100, 128),
@@ -114,6 +119,9 @@ def test_misaligned_pointers_rejected(lib):
                                     None) == E_ALIGN
     assert lib.fp8bw_quantize_weight_block_pow2(A, 128, 128, B, C, D + 8,
                                                 None) == E_ALIGN
+    assert lib.fp8bw_gemm_fprop_quant(A, B, C, D, 128, 128, 128, E,
+                                      E + 0x100008, E + 0x200000,
+                                      None) == E_ALIGN
 
 
 def test_aliased_outputs_rejected(lib):
@@ -124,6 +132,9 @@ def test_aliased_outputs_rejected(lib):
                                 None) == E_ALIAS
     assert lib.fp8bw_gemm_wgrad(A, B, C, D, 128, 128, 128, C + 256,
                                 None) == E_ALIAS
+    # fused quantisation: codes on top of the bf16 output
+    assert lib.fp8bw_gemm_fprop_quant(A, B, C, D, 128, 128, 128, E, E + 64,
+                                      E + 0x100000, None) == E_ALIAS
     # the fp32 dW is 4 bytes per element: [C - 128*128*4 + 16, C + 16)
     # reaches into qX^T at C
     assert lib.fp8bw_gemm_wgrad_f32(A, B, C, D, 128, 128, 128,
