@@ -317,6 +317,21 @@ int launch_gemm_pow2(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t s
   return cudaGetLastError() == cudaSuccess ? FP8BW_OK : FP8BW_ERR_LAUNCH;
 }
 
+// One block whose thread 0 waits, with the library's bounded wait, on an
+// mbarrier phase that nothing completes; the wait gives up after limit_ns and
+// records a timeout exactly as the kernels' waits do.
+__global__ void wait_selftest_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0u;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0u, &abort_flag, kErrTimeoutEpi, limit_ns);
+}
+
 int run_gemm(const GemmProblem& p, cudaStream_t stream) {
   DeviceInfo dev;
   int st = current_device_info(&dev);
@@ -362,7 +377,7 @@ using namespace fp8bw;
 
 extern "C" {
 
-int fp8bw_version(void) { return 103; }
+int fp8bw_version(void) { return 104; }
 
 const char* fp8bw_status_string(int status) {
   switch (status) {
@@ -665,6 +680,16 @@ int fp8bw_gemm_wgrad_f32(const uint8_t* qdy_t, const float* sdy_t, const uint8_t
                          int accumulate, void* stream) {
   return wgrad_common(qdy_t, sdy_t, qx_t, sx_t, m, n, k, dw,
                       accumulate ? gemm::kOutF32Add : gemm::kOutF32, false, stream);
+}
+
+int fp8bw_selftest_wait_timeout(int64_t limit_ns, void* stream) {
+  if (limit_ns < 0 || limit_ns > 1000000000) return FP8BW_ERR_SHAPE;
+  DeviceInfo dev;
+  int st = current_device_info(&dev);
+  if (st != FP8BW_OK) return st;
+  wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(limit_ns));
+  return cudaGetLastError() == cudaSuccess ? FP8BW_OK : FP8BW_ERR_LAUNCH;
 }
 
 int fp8bw_check_device_error(void* stream) {

@@ -97,18 +97,20 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 constexpr uint32_t kWaitSliceNs = 1000000u;
 
 // Wait for the phase with the given parity to complete. Gives up (returns
-// false) when *abort becomes non-zero or after kWaitLimitNs; on a timeout it
+// false) when *abort becomes non-zero or after limit_ns (default
+// kWaitLimitNs); on a timeout it
 // records `err_bit` in the device error word and raises *abort so that the
 // other warps of the CTA stop waiting too.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           volatile uint32_t* abort,
-                                          uint32_t err_bit) {
+                                          uint32_t err_bit,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
     if (mbar_try_wait_sleep(bar, parity, kWaitSliceNs)) return true;
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       atomicOr(&g_device_error, err_bit);
       *abort = 1u;
       return false;

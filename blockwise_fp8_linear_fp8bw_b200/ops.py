@@ -197,6 +197,11 @@ def fp8bw_gemm_dgrad_quant(qdy, sdy, qw, qw_is_transposed, sw, dx, qdx, sdx,
            "fp8bw_gemm_dgrad_quant")
 
 
+def fp8bw_selftest_wait_timeout(limit_ns, stream=None):
+    _check(_lib.fp8bw_selftest_wait_timeout(int(limit_ns), _stream(stream)),
+           "fp8bw_selftest_wait_timeout")
+
+
 def fp8bw_check_device_error(stream=None):
     _check(_lib.fp8bw_check_device_error(_stream(stream)),
            "fp8bw_check_device_error")

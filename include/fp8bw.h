@@ -228,6 +228,15 @@ int fp8bw_gemm_wgrad_pow2(const uint8_t* qdy_t, const float* sdy_t,
  * the synchronisation itself failed). */
 int fp8bw_check_device_error(void* stream);
 
+/* Test of the error path of the library's bounded device-side waits: one
+ * block waits on a barrier that nothing completes; after limit_ns (0 to 1e9
+ * ns, else FP8BW_ERR_SHAPE) the wait gives up and records a timeout, so the
+ * next fp8bw_check_device_error returns FP8BW_ERR_DEVICE_TIMEOUT (and clears
+ * it). Nothing faults or hangs; the context stays usable. Writes nothing but
+ * the error record. (No counterpart on the pages: robustness of this
+ * library.) */
+int fp8bw_selftest_wait_timeout(int64_t limit_ns, void* stream);
+
 /* Static, NUL-terminated description of a status code. */
 const char* fp8bw_status_string(int status);
 

@@ -37,14 +37,14 @@ def lib():
 
 def test_every_declared_symbol_is_exported(lib):
     names = declared_functions()
-    assert len(names) == 18
+    assert len(names) == 19
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(_native.SIGNATURES)
 
 
 def test_status_strings_and_version(lib):
-    assert lib.fp8bw_version() == 103
+    assert lib.fp8bw_version() == 104
     for st in (OK, E_NULL, E_SHAPE, E_ALIGN, E_DEVICE, E_LAUNCH, E_TIMEOUT,
                E_CUDA, E_ALIAS, E_SCALE):
         s = lib.fp8bw_status_string(st).decode()
@@ -79,6 +79,11 @@ def test_null_pointers_rejected(lib):
                                       E + 0x100000, None) == E_NULL
     assert lib.fp8bw_gemm_dgrad_quant(A, B, C, 1, D, 128, 128, 128, E,
                                       E + 0x100000, None, None) == E_NULL
+
+
+def test_selftest_limit_checked(lib):
+    assert lib.fp8bw_selftest_wait_timeout(-1, None) == E_SHAPE
+    assert lib.fp8bw_selftest_wait_timeout(2 * 10**9, None) == E_SHAPE
 
 
 @pytest.mark.parametrize("rows,cols", [(-16, 128), (128, -16), (100, 128),
