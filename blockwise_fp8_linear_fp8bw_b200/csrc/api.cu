@@ -402,7 +402,9 @@ namespace {
 
 int quantize_rowwise(bool pow2, const uint16_t* x, int64_t rows, int64_t cols, uint8_t* q,
                      float* s, void* stream) {
-  if (!dim_ok(rows) || !dim_ok(cols) || cdiv(rows, 128) > 65535) return FP8BW_ERR_SHAPE;
+  if (!dim_ok(rows) || !dim_ok(cols) || cdiv(rows, 128) > 65535 ||
+      cdiv(rows, 128) * cdiv(cols, 128) > INT32_MAX)
+    return FP8BW_ERR_SHAPE;
   if (missing(x, rows * cols) || missing(q, rows * cols) || missing(s, cdiv(cols, 128) * rows))
     return FP8BW_ERR_NULL;
   if (!aligned16(x) || !aligned16(q) || !aligned16(s)) return FP8BW_ERR_ALIGN;
@@ -419,7 +421,9 @@ int quantize_rowwise(bool pow2, const uint16_t* x, int64_t rows, int64_t cols, u
 
 int quantize_colwise(bool pow2, const uint16_t* x, int64_t rows, int64_t cols, uint8_t* q_t,
                      float* s_t, uint8_t* q_row, float* s_row, void* stream) {
-  if (!dim_ok(rows) || !dim_ok(cols) || cdiv(rows, 128) > 65535) return FP8BW_ERR_SHAPE;
+  if (!dim_ok(rows) || !dim_ok(cols) || cdiv(rows, 128) > 65535 ||
+      cdiv(rows, 128) * cdiv(cols, 128) > INT32_MAX)
+    return FP8BW_ERR_SHAPE;
   if (missing(x, rows * cols) || missing(q_t, rows * cols) || missing(s_t, cdiv(rows, 128) * cols))
     return FP8BW_ERR_NULL;
   if (rows * cols > 0 && (q_row == nullptr) != (s_row == nullptr)) return FP8BW_ERR_NULL;
@@ -443,7 +447,9 @@ int quantize_colwise(bool pow2, const uint16_t* x, int64_t rows, int64_t cols, u
 
 int quantize_weight_block(bool pow2, const uint16_t* w, int64_t n, int64_t k, uint8_t* q,
                           float* s, uint8_t* q_t, void* stream) {
-  if (!dim_ok(n) || !dim_ok(k) || cdiv(n, 128) > 65535) return FP8BW_ERR_SHAPE;
+  if (!dim_ok(n) || !dim_ok(k) || cdiv(n, 128) > 65535 ||
+      cdiv(n, 128) * cdiv(k, 128) > INT32_MAX)
+    return FP8BW_ERR_SHAPE;
   if (missing(w, n * k) || missing(q, n * k) || missing(s, cdiv(n, 128) * cdiv(k, 128)))
     return FP8BW_ERR_NULL;
   if (!aligned16(w) || !aligned16(q) || !aligned16(s) || !aligned16(q_t)) return FP8BW_ERR_ALIGN;

@@ -31,6 +31,9 @@
  *   - Every call is asynchronous on `stream` (a cudaStream_t, NULL = legacy
  *     default stream) and returns an fp8bw_status. Argument errors are found
  *     on the host before anything is launched, and then nothing is written.
+ *   - Limits: every dimension <= 2^30; a quantiser takes at most 65535 row
+ *     tiles of 128 and fewer than 2^31 tiles of 128 x 128; a GEMM at most 2^30
+ *     output tiles of 256 x 256 (else FP8BW_ERR_SHAPE).
  *   - Shapes: every dimension >= 0 and a multiple of 16. Dimensions that are
  *     not multiples of 128 give a short last group (its amax runs over the
  *     elements present) and a short last chunk. A zero dimension is a no-op,

@@ -81,6 +81,15 @@ def test_null_pointers_rejected(lib):
                                       E + 0x100000, None, None) == E_NULL
 
 
+def test_tile_count_limit(lib):
+    rows, cols = 65535 * 128, 1 << 30          # 65535 * 2^23 tiles of 128x128
+    assert lib.fp8bw_quantize_rowwise(A, rows, cols, B, C, None) == E_SHAPE
+    assert lib.fp8bw_quantize_colwise(A, rows, cols, B, C, None, None,
+                                      None) == E_SHAPE
+    assert lib.fp8bw_quantize_weight_block(A, rows, cols, B, C, None,
+                                           None) == E_SHAPE
+
+
 def test_selftest_limit_checked(lib):
     assert lib.fp8bw_selftest_wait_timeout(-1, None) == E_SHAPE
     assert lib.fp8bw_selftest_wait_timeout(2 * 10**9, None) == E_SHAPE
