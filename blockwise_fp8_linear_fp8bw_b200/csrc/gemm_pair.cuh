@@ -47,7 +47,9 @@
 //               by box, and writes it with TMA: bf16 32x32 boxes (the GEMM's
 //               output), or fp32 16-column x 32-row boxes, either stored or
 //               added element-wise into the fp32 tensor already in memory
-//               (a weight-gradient accumulator).
+//               (a weight-gradient accumulator); in block mode the bf16 output
+//               can also leave with its own row-wise E4M3 codes and scales
+//               (one thread's 128 columns of its row are one 1x128 group).
 // With BN = 256 the producer warps give registers to the promotion warps
 // (setmaxnreg 56 / 224: 4*32*56 + 8*32*224 = 384 * 168, the launch budget).
 // Every mbarrier wait is bounded (about 2 s, common.cuh); on expiry the CTA
