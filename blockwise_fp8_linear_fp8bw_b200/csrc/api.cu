@@ -40,6 +40,11 @@ int current_device_info(DeviceInfo* out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
     return FP8BW_ERR_DEVICE;
+  // The tensor-map encoder is a driver call and needs the device's context
+  // current on this thread; a thread that has so far only reused cached
+  // allocations (autograd's backward thread, for one) may not have it yet.
+  // cudaSetDevice makes the primary context current.
+  if (cudaSetDevice(dev) != cudaSuccess) return FP8BW_ERR_DEVICE;
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceInfo& d = g_dev[dev];
   if (d.checked == 0) {

@@ -1,0 +1,106 @@
+"""A training linear layer on the library's blockwise-FP8 path.
+
+Y = X W^T with the E4M3 quantisers and GEMMs of this library (Puro-2B report:
+arxiv-wiki summary, "Approach" item (4) -- E4M3, 1x128 activation groups,
+128x128 weight blocks; paperlayer.ai summary, Appendix C, "FP8 implementation
+pipeline" -- forward, data-gradient and weight-gradient GEMMs in E4M3, bf16
+hidden flow, fp32 gradients):
+
+  forward   W -> 128x128 block codes (+ transposed codes for dgrad)
+            X -> row-wise (fprop) and column-wise (wgrad) codes, one pass
+            Y = fprop(X, W)                                        bf16
+  backward  dY -> row-wise (dgrad) and column-wise (wgrad) codes, one pass
+            dX = dgrad(dY, W)                                      bf16
+            dW = wgrad(dY, X): added in fp32 into weight.main_grad when the
+                 weight carries one (gradient accumulation over
+                 micro-batches), else returned in the weight's dtype
+
+Every step runs in the CUDA library; this module only reshapes tensors and
+keeps the codes the backward pass needs. Inputs must be bf16 CUDA tensors
+whose dimensions are multiples of 16.
+"""
+import torch
+
+from . import ops
+
+
+def _rows(t, k):
+    if not t.is_cuda or t.dtype != torch.bfloat16:
+        raise ValueError("expected a bf16 CUDA tensor, got %s on %s"
+                         % (t.dtype, t.device))
+    return t.reshape(-1, k).contiguous()
+
+
+class BlockwiseFp8LinearFunction(torch.autograd.Function):
+    """y = x @ weight.T on the blockwise-FP8 path (see the module docstring).
+    `pow2` selects the power-of-two-scale variant."""
+
+    @staticmethod
+    def forward(ctx, x, weight, pow2=False):
+        n, k = weight.shape
+        x2 = _rows(x, k)
+        w = _rows(weight, k)
+        qw, sw, qw_t = ops.quantize_weight_block(w, transposed=True, pow2=pow2)
+        qx_t, sx_t, qx, sx = ops.quantize_colwise(x2, with_rowwise=True,
+                                                  pow2=pow2)
+        y = ops.gemm_fprop(qx, sx, qw, sw, pow2=pow2)
+        ctx.save_for_backward(qx_t, sx_t, qw_t, sw)
+        ctx.pow2 = pow2
+        ctx.weight = weight
+        ctx.x_shape = x.shape
+        return y.reshape(*x.shape[:-1], n)
+
+    @staticmethod
+    def backward(ctx, dy):
+        qx_t, sx_t, qw_t, sw = ctx.saved_tensors
+        weight = ctx.weight
+        n, k = weight.shape
+        dy2 = _rows(dy, n)
+        qdy_t, sdy_t, qdy, sdy = ops.quantize_colwise(dy2, with_rowwise=True,
+                                                      pow2=ctx.pow2)
+        dx = dw = None
+        if ctx.needs_input_grad[0]:
+            dx = ops.gemm_dgrad(qdy, sdy, qw_t, sw, qw_is_transposed=True,
+                                pow2=ctx.pow2).reshape(ctx.x_shape)
+        if ctx.needs_input_grad[1]:
+            main = getattr(weight, "main_grad", None)
+            if main is not None and not ctx.pow2:
+                ops.gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, main_grad=main)
+            elif main is not None:
+                main += ops.gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t,
+                                       pow2=True).float()
+            else:
+                dw = ops.gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t, pow2=ctx.pow2)
+                if dw.dtype != weight.dtype:
+                    dw = dw.to(weight.dtype)
+        return dx, dw, None
+
+
+class BlockwiseFp8Linear(torch.nn.Module):
+    """Bias-free linear layer (in_features -> out_features) whose three GEMMs
+    run in blockwise E4M3. The weight is a bf16 parameter [out, in]; give it
+    an fp32 `main_grad` tensor of the same shape to have dW accumulated there
+    in fp32 instead of returned as `weight.grad`."""
+
+    def __init__(self, in_features, out_features, device=None, pow2=False):
+        super().__init__()
+        if in_features % 16 or out_features % 16:
+            raise ValueError("in_features and out_features must be multiples "
+                             "of 16")
+        self.in_features = in_features
+        self.out_features = out_features
+        self.pow2 = pow2
+        w = torch.empty((out_features, in_features), dtype=torch.bfloat16,
+                        device=device)
+        torch.nn.init.normal_(w, std=0.02)
+        self.weight = torch.nn.Parameter(w)
+
+    def forward(self, x):
+        return BlockwiseFp8LinearFunction.apply(x, self.weight, self.pow2)
+
+    def extra_repr(self):
+        return "in_features=%d, out_features=%d, pow2=%s" % (
+            self.in_features, self.out_features, self.pow2)
+
+
+__all__ = ["BlockwiseFp8Linear", "BlockwiseFp8LinearFunction"]
