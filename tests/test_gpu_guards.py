@@ -1,0 +1,126 @@
+"""Out-of-bounds writes and unwritten outputs (in place of a memory checker):
+every output of every entry point is placed in a larger buffer filled with
+0xCD, 4 KB of guard bytes on each side; after the call the guards must be
+untouched and the output must equal the result of a normal call (whose values
+the parity tests check against the oracle) -- so every byte was written, and
+nothing outside it. Ragged shapes."""
+import pytest
+
+import synthetic as S
+from helpers import bf16_np_to_torch
+
+pytestmark = pytest.mark.gpu
+
+GUARD = 4096
+SHAPES = [(272, 400, 528), (16, 16, 16), (1040, 272, 144), (384, 1296, 640)]
+
+
+def _ops():
+    from blockwise_fp8_linear_fp8bw_b200 import ops
+    return ops
+
+
+class Guarded:
+    """Output tensors carved out of one poisoned byte buffer."""
+
+    def __init__(self):
+        self.parts = []
+
+    def make(self, shape, dtype):
+        import torch
+        n = 1
+        for d in shape:
+            n *= d
+        nbytes = n * torch.empty((), dtype=dtype).element_size()
+        buf = torch.full((GUARD + nbytes + GUARD,), 0xCD, dtype=torch.uint8, device="cuda")
+        t = buf[GUARD:GUARD + nbytes].view(dtype).view(shape)
+        self.parts.append((buf, nbytes))
+        return t
+
+    def check(self, what):
+        import torch
+        torch.cuda.synchronize()
+        for buf, nbytes in self.parts:
+            head, tail = buf[:GUARD], buf[GUARD + nbytes:]
+            assert bool((head == 0xCD).all()) and bool((tail == 0xCD).all()), \
+                what + ": a write outside the output"
+
+
+def _eq(a, b):
+    import torch
+    return torch.equal(a.view(torch.uint8), b.view(torch.uint8))
+
+
+@pytest.mark.parametrize("m,n,k", SHAPES)
+@pytest.mark.parametrize("pow2", [False, True])
+def test_quantisers_write_exactly_their_outputs(m, n, k, pow2):
+    import torch
+    ops = _ops()
+    x = bf16_np_to_torch(S.bf16_normal((m, k), 0, 970, **S.X_DIST))
+    w = bf16_np_to_torch(S.bf16_normal((n, k), 0, 971, **S.W_DIST))
+    cd = lambda a: (a + 127) // 128  # noqa: E731
+    g = Guarded()
+    q, s = g.make((m, k), torch.uint8), g.make((cd(k), m), torch.float32)
+    q_t, s_t = g.make((k, m), torch.uint8), g.make((cd(m), k), torch.float32)
+    q2, s2 = g.make((m, k), torch.uint8), g.make((cd(k), m), torch.float32)
+    qw, sw, qw_t = (g.make((n, k), torch.uint8), g.make((cd(n), cd(k)), torch.float32),
+                    g.make((k, n), torch.uint8))
+    ops.fp8bw_quantize_rowwise(x, q, s, pow2=pow2)
+    ops.fp8bw_quantize_colwise(x, q_t, s_t, q2, s2, pow2=pow2)
+    ops.fp8bw_quantize_weight_block(w, qw, sw, qw_t, pow2=pow2)
+    g.check("quantisers")
+    rq, rs = ops.quantize_rowwise(x, pow2=pow2)
+    rq_t, rs_t = ops.quantize_colwise(x, pow2=pow2)
+    rqw, rsw, rqw_t = ops.quantize_weight_block(w, pow2=pow2)
+    assert _eq(q, rq) and _eq(s, rs) and _eq(q2, rq) and _eq(s2, rs)
+    assert _eq(q_t, rq_t) and _eq(s_t, rs_t)
+    assert _eq(qw, rqw) and _eq(sw, rsw) and _eq(qw_t, rqw_t)
+
+
+@pytest.mark.parametrize("m,n,k", SHAPES)
+def test_gemms_write_exactly_their_outputs(m, n, k):
+    import torch
+    ops = _ops()
+    x = bf16_np_to_torch(S.bf16_normal((m, k), 0, 980, **S.X_DIST))
+    w = bf16_np_to_torch(S.bf16_normal((n, k), 0, 981, **S.W_DIST))
+    dy = bf16_np_to_torch(S.bf16_normal((m, n), 0, 982, **S.DY_DIST))
+    cd = lambda a: (a + 127) // 128  # noqa: E731
+    for pow2 in (False, True):
+        qx_t, sx_t, qx, sx = ops.quantize_colwise(x, with_rowwise=True, pow2=pow2)
+        qdy_t, sdy_t, qdy, sdy = ops.quantize_colwise(dy, with_rowwise=True, pow2=pow2)
+        qw, sw, qw_t = ops.quantize_weight_block(w, pow2=pow2)
+        g = Guarded()
+        y, dx, dx2, dw = (g.make((m, n), torch.bfloat16), g.make((m, k), torch.bfloat16),
+                          g.make((m, k), torch.bfloat16), g.make((n, k), torch.bfloat16))
+        ops.fp8bw_gemm_fprop(qx, sx, qw, sw, y, pow2=pow2)
+        ops.fp8bw_gemm_dgrad(qdy, sdy, qw_t, 1, sw, dx, pow2=pow2)
+        ops.fp8bw_gemm_dgrad(qdy, sdy, qw, 0, sw, dx2, pow2=pow2)
+        ops.fp8bw_gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t, dw, pow2=pow2)
+        g.check("GEMMs pow2=%s" % pow2)
+        assert _eq(y, ops.gemm_fprop(qx, sx, qw, sw, pow2=pow2))
+        ref_dx = ops.gemm_dgrad(qdy, sdy, qw_t, sw, pow2=pow2)
+        assert _eq(dx, ref_dx) and _eq(dx2, ops.gemm_dgrad(qdy, sdy, qw, sw, False, pow2=pow2))
+        assert _eq(dw, ops.gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t, pow2=pow2))
+    # fp32 wgrad (store and add) and the fused-quantisation outputs
+    qx_t, sx_t, qx, sx = ops.quantize_colwise(x, with_rowwise=True)
+    qdy_t, sdy_t, qdy, sdy = ops.quantize_colwise(dy, with_rowwise=True)
+    qw, sw, qw_t = ops.quantize_weight_block(w)
+    g = Guarded()
+    dw32 = g.make((n, k), torch.float32)
+    acc32 = g.make((n, k), torch.float32)
+    y, qy, sy = g.make((m, n), torch.bfloat16), g.make((m, n), torch.uint8), \
+        g.make((cd(n), m), torch.float32)
+    dx, qdx, sdx = g.make((m, k), torch.bfloat16), g.make((m, k), torch.uint8), \
+        g.make((cd(k), m), torch.float32)
+    acc32.zero_()
+    ops.fp8bw_gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, dw32)
+    ops.fp8bw_gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, acc32, accumulate=True)
+    ops.fp8bw_gemm_fprop_quant(qx, sx, qw, sw, y, qy, sy)
+    ops.fp8bw_gemm_dgrad_quant(qdy, sdy, qw_t, 1, sw, dx, qdx, sdx)
+    g.check("fp32 wgrad and fused quantisation")
+    ref32 = ops.gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t)
+    assert _eq(dw32, ref32) and _eq(acc32, ref32)     # 0 + P == P exactly
+    ry, rqy, rsy = ops.gemm_fprop_quant(qx, sx, qw, sw)
+    rdx, rqdx, rsdx = ops.gemm_dgrad_quant(qdy, sdy, qw_t, sw)
+    assert _eq(y, ry) and _eq(qy, rqy) and _eq(sy, rsy)
+    assert _eq(dx, rdx) and _eq(qdx, rqdx) and _eq(sdx, rsdx)
