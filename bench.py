@@ -453,7 +453,9 @@ def time_next_rows(o, bufs, stream, warmup, rounds):
 
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,"
+    """nvidia-smi samples every 200 ms; stop() summarises those taken inside
+    the timed window (all of them if none fell inside)."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,"
               "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,"
@@ -470,7 +472,8 @@ class ClockSampler:
         except Exception:
             self.proc = None
 
-    def stop(self):
+    def stop(self, window=None):
+        """window: (start, end) in time.time() seconds of the timed region."""
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -479,26 +482,39 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
             out, _ = self.proc.communicate()
-        mhz, maxes, reasons = [], [], set()
+        return self.summarise(out, window)
+
+    @staticmethod
+    def summarise(out, window=None):
+        import datetime
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
                  "sw_power_cap"]
+        rows = []
         for line in out.splitlines():
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
                 continue
             try:
-                mhz.append(float(parts[1]))
-                maxes.append(float(parts[2]))
+                ts = datetime.datetime.strptime(
+                    parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                ts = None
+            try:
+                rows.append((ts, float(parts[2]), float(parts[3]),
+                             [n for n, v in zip(names, parts[6:10])
+                              if v.lower().startswith("active")]))
             except ValueError:
                 continue
-            for name, val in zip(names, parts[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
-        if not mhz:
+        if window is not None:
+            inside = [r for r in rows
+                      if r[0] is not None and window[0] <= r[0] <= window[1]]
+            rows = inside or rows
+        if not rows:
             return None
-        return {"sm_mhz": statistics.median(mhz),
-                "sm_max_mhz": max(maxes) if maxes else None,
-                "reasons": sorted(reasons), "samples": len(mhz)}
+        return {"sm_mhz": statistics.median(r[1] for r in rows),
+                "sm_max_mhz": max(r[2] for r in rows),
+                "reasons": sorted({n for r in rows for n in r[3]}),
+                "samples": len(rows)}
 
 
 def gpu_uuid(torch, dev):
@@ -562,14 +578,16 @@ def run_gpu(args):
     time.sleep(0.6)
     barrier()
     torch.cuda.synchronize()
+    wall0 = time.time()
     with torch.cuda.stream(stream):
         t_start.record(stream)
         for s in range(args.steps):
             run_step(events if s == args.steps - 1 else None)
         t_end.record(stream)
     torch.cuda.synchronize()
+    wall1 = time.time()
     barrier()
-    clk = clocks.stop()
+    clk = clocks.stop((wall0, wall1))
     o.fp8bw_check_device_error(stream)
     ms = max_over_ranks(t_start.elapsed_time(t_end) / args.steps, world, dev)
 
