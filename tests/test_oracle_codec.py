@@ -50,6 +50,25 @@ def test_encode_random_fp32_patterns_match_torch():
     assert np.array_equal(oracle.e4m3_encode(f), _torch_encode(f))
 
 
+def test_encode_every_fp32_in_the_rounding_range_matches_torch():
+    # Every fp32 bit pattern with 2^-12 <= |t| <= 464, both signs: all the
+    # rounding decisions of the format (the smallest one is at 2^-10).
+    # Below 2^-12 every value must give a signed zero.
+    lo = int(np.float32(2.0 ** -12).view(np.uint32))
+    hi = int(np.float32(464.0).view(np.uint32))
+    step = 1 << 24
+    for start in range(lo, hi + 1, step):
+        bits = np.arange(start, min(start + step, hi + 1), dtype=np.uint32)
+        for sign in (0, 0x80000000):
+            f = (bits | np.uint32(sign)).view(np.float32)
+            assert np.array_equal(oracle.e4m3_encode(f), _torch_encode(f)), \
+                hex(start | sign)
+    tiny = np.arange(0, lo, 997, dtype=np.uint32)
+    for sign, code in ((0, 0x00), (0x80000000, 0x80)):
+        f = (tiny | np.uint32(sign)).view(np.float32)
+        assert np.all(oracle.e4m3_encode(f) == code)
+
+
 def test_encode_midpoints_and_neighbours_match_torch():
     # All midpoints between adjacent E4M3 magnitudes, and the fp32 values one
     # ulp either side of each: the rounding decision points.
