@@ -165,3 +165,55 @@ def test_valid_call_without_device_reports_device_error(lib):
                                 None) == E_DEVICE
     assert lib.fp8bw_gemm_wgrad_f32(A, B, C, D, 128, 128, 128, E, 1,
                                     None) == E_DEVICE
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "fp8bw.h"
+
+typedef int (*gemm_fn)(const uint8_t*, const float*, const uint8_t*,
+                       const float*, int64_t, int64_t, int64_t, uint16_t*,
+                       void*);
+
+int main(void) {
+    gemm_fn f = fp8bw_gemm_fprop;
+    uint8_t code = 0;
+    float scale = 1.0f;
+    uint16_t out = 0;
+    /* no device needed: the null operand is rejected on the host */
+    int st = f(NULL, &scale, &code, &scale, 128, 128, 128, &out, NULL);
+    printf("%d %d %s|%s\n", fp8bw_version(), st, fp8bw_status_string(st),
+           fp8bw_status_string(FP8BW_OK));
+    return (st == FP8BW_ERR_NULL && out == 0) ? 0 : 1;
+}
+"""
+
+
+@pytest.mark.parametrize("compiler,std", [("gcc", "-std=c11"),
+                                          ("g++", "-std=c++17")])
+def test_header_builds_a_plain_client(lib, tmp_path, compiler, std):
+    """include/fp8bw.h is self-contained C: a C11 (and a C++17) program that
+    includes it builds with -pedantic -Werror, links against libfp8bw.so and
+    gets the host-side answers (version, status strings, a rejected call)."""
+    import shutil
+    import subprocess
+    if shutil.which(compiler) is None:
+        pytest.skip(compiler + " not available")
+    src = tmp_path / ("client.c" if compiler == "gcc" else "client.cpp")
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(_native.LIB_PATH)
+    cmd = [compiler, std, "-Wall", "-Wextra", "-pedantic", "-Werror",
+           "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+           "-L", libdir, "-l:" + os.path.basename(_native.LIB_PATH),
+           "-Wl,-rpath," + libdir]
+    subprocess.run(cmd, check=True, capture_output=True, text=True)
+    run = subprocess.run([str(exe)], capture_output=True, text=True,
+                         timeout=60)
+    assert run.returncode == 0, run.stdout + run.stderr
+    version, status, rest = run.stdout.strip().split(" ", 2)
+    assert int(version) == lib.fp8bw_version() and int(status) == E_NULL
+    null_msg, ok_msg = rest.split("|")
+    assert null_msg == lib.fp8bw_status_string(E_NULL).decode()
+    assert ok_msg == lib.fp8bw_status_string(OK).decode()
