@@ -13,7 +13,9 @@ hidden flow, fp32 gradients):
             dX = dgrad(dY, W)                                      bf16
             dW = wgrad(dY, X): added in fp32 into weight.main_grad when the
                  weight carries one (gradient accumulation over
-                 micro-batches), else returned in the weight's dtype
+                 micro-batches), else returned in the weight's dtype.
+                 The power-of-two-scale wgrad writes bf16 only, so on that
+                 path the bf16 dW is widened and then added to main_grad.
 
 Every step runs in the CUDA library; this module only reshapes tensors and
 keeps the codes the backward pass needs. Inputs must be bf16 CUDA tensors
