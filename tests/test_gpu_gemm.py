@@ -4,9 +4,10 @@ propagation, data-gradient and weight-gradient), through the C ABI.
 
 Each output element must satisfy |y - ref| <= 1e-3 * sum_k |a_k b_k| + 1 bf16
 ulp(ref), where ref is the oracle's fp64 value and the sum runs over the
-dequantised operands. Small cases compare every element; full-size cases
-compare >= 16 seeded points per 128x128 output tile plus two full rows and
-two full columns, in the launch configuration the benchmark uses."""
+dequantised operands. Small cases and the 8192 x 4096 x 2048 fprop compare
+every element; the larger full-size cases compare >= 16 seeded points per
+128x128 output tile plus two full rows and two full columns, in the launch
+configuration the benchmark uses."""
 import numpy as np
 import pytest
 
@@ -118,8 +119,8 @@ def test_empty_contraction_writes_zeros():
     assert torch.count_nonzero(y).item() == 0
 
 
-def test_full_size_qkv_fprop():
-    _fprop_case(8192, 4096, 2048, S.tensor_id("qkv", "x"), full=False)
+def test_full_size_qkv_fprop_every_element():
+    _fprop_case(8192, 4096, 2048, S.tensor_id("qkv", "x"), full=True)
 
 
 def test_full_size_mlp_fprop():
@@ -134,6 +135,18 @@ def test_full_size_mlp_backward():
     _dgrad_case(16384, 12288, 2048, S.tensor_id("gate_up", "dy"), True,
                 full=False)
     _wgrad_case(16384, 12288, 2048, S.tensor_id("gate_up", "dy"), full=False)
+    _ops().fp8bw_check_device_error()
+
+
+@pytest.mark.parametrize("kind", ["qkv", "o"])
+def test_full_size_attention_linears(kind):
+    """The QKV and O linears of the 28-layer stack at M = 16384 (the MLP
+    linears are covered above): fprop, dgrad on transposed weight codes and
+    wgrad, each on its own draws."""
+    k, n = S.LINEARS[kind]
+    _fprop_case(16384, n, k, S.tensor_id(kind, "x", 0), full=False)
+    _dgrad_case(16384, n, k, S.tensor_id(kind, "dy", 0), True, full=False)
+    _wgrad_case(16384, n, k, S.tensor_id(kind, "dy", 0), full=False)
     _ops().fp8bw_check_device_error()
 
 

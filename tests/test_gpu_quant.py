@@ -119,6 +119,18 @@ FULL = {
 }
 
 
+@pytest.mark.parametrize("kind", ["qkv", "o"])
+def test_full_size_attention_quantisers(kind):
+    """Every element of the 28-layer stack's QKV and O inputs, output
+    gradients (row + column, one pass) and weights at M = 16384."""
+    lin = [l for l in S.workload("stack28_m16384")
+           if l.kind == kind and l.layer == 0][0]
+    _check_colwise(S.draw_x(lin), True)
+    _check_colwise(S.draw_dy(lin), True)
+    _check_weight(S.draw_w(lin))
+    _ops().fp8bw_check_device_error()
+
+
 @pytest.mark.parametrize("name", sorted(FULL))
 def test_full_size_activation_quantisers(name):
     """Every element of the workloads' activations and gradients, row-wise and
