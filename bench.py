@@ -313,12 +313,22 @@ class LinearBuffers:
         ]
 
 
+def linear_names(kinds):
+    """'QKV, O, gate/up and down' for the linear kinds given, in order."""
+    label = {"qkv": "QKV", "o": "O", "gate_up": "gate/up", "down": "down"}
+    names = [label.get(k, k) for k in kinds]
+    if len(names) < 2:
+        return "".join(names)
+    return ", ".join(names[:-1]) + " and " + names[-1]
+
+
 def time_next_rows(o, bufs, stream, warmup, rounds):
     """Rows beyond the step, timed after it on the same buffers (not part of
     `value`): wgrad with an fp32 dW added into an fp32 main-grad buffer, the
     four linears of a layer in turn (their operands together exceed L2)."""
     import torch
     dev = bufs[0].qx_t.device
+    names = linear_names([b.kind for b in bufs])
     grads = [torch.zeros((b.n, b.k), dtype=torch.float32, device=dev)
              for b in bufs]
     calls = [(2 * TOKENS * b.n * b.k,
@@ -346,8 +356,8 @@ def time_next_rows(o, bufs, stream, warmup, rounds):
     out = {"wgrad_f32_accumulate": {
         "achieved": flop / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
         "launches": rounds * len(calls), "avg_launch_ms": ms / (rounds * len(calls)),
-        "what": "dW (fp32) += dY^T X for the QKV, O, gate/up and down "
-                "linears at M=%d, in turn; timed after the step" % TOKENS}}
+        "what": "dW (fp32) += dY^T X for the %s linears at M=%d, in turn; "
+                "timed after the step" % (names, TOKENS)}}
 
     # fprop and dgrad that also quantise their own bf16 output row-wise,
     # against the same GEMMs followed by the row-wise quantiser.
@@ -398,10 +408,10 @@ def time_next_rows(o, bufs, stream, warmup, rounds):
         "achieved": gfl / (t_f * 1e-3) / 1e12, "unit": "TFLOP/s",
         "ms_fused": t_f, "ms_gemm_then_quantiser": t_u,
         "saved_frac": 1.0 - t_f / t_u,
-        "what": "fprop and dgrad of the four linears (M=%d) writing bf16 "
+        "what": "fprop and dgrad of the %s linears (M=%d) writing bf16 "
                 "plus the row-wise E4M3 codes and scales of that output, "
                 "against the same GEMMs followed by the row-wise quantiser; "
-                "timed after the step" % TOKENS}
+                "timed after the step" % (names, TOKENS)}
     del qy, sy, qdx, sdx
 
     # The whole step again with power-of-two scales (quantisers and GEMMs on
@@ -446,9 +456,9 @@ def time_next_rows(o, bufs, stream, warmup, rounds):
                            else u / (ms_ * 1e-3) / 1e9)
                       for kk, (ms_, u) in kinds_.items()},
         "breakdown_units": "gemm_*: TFLOP/s, quant_*: GB/s",
-        "what": "the same 28-layer step with power-of-two scales (s = 2^E, "
+        "what": "the same %d-layer step with power-of-two scales (s = 2^E, "
                 "the smallest E with 448*2^E >= amax) applied by the tensor "
-                "cores' UE8M0 block scaling; timed after the step"}
+                "cores' UE8M0 block scaling; timed after the step" % LAYERS}
     return out
 
 

@@ -40,3 +40,10 @@ def test_clock_summary_without_timestamps():
     line = "n/a, 0, 1700, 1965, 900.0, 0x0, Not Active, Not Active, Not Active, Not Active"
     s = bench.ClockSampler.summarise("\n".join([line] * 3), (0.0, 1.0))
     assert s["samples"] == 3 and s["sm_mhz"] == 1700 and s["reasons"] == []
+
+
+def test_linear_names():
+    assert bench.linear_names(["qkv", "o", "gate_up", "down"]) == \
+        "QKV, O, gate/up and down"
+    assert bench.linear_names(["gate_up"]) == "gate/up"
+    assert bench.linear_names(["o", "down"]) == "O and down"
