@@ -47,3 +47,70 @@ def test_linear_names():
         "QKV, O, gate/up and down"
     assert bench.linear_names(["gate_up"]) == "gate/up"
     assert bench.linear_names(["o", "down"]) == "O and down"
+
+
+class _FakeEvent:
+    def __init__(self, enable_timing=False):
+        pass
+
+    def record(self, stream=None):
+        pass
+
+    def elapsed_time(self, other):
+        return 2.0
+
+
+class _FakeLibrary:
+    """Every entry point of the binding does nothing and counts the call."""
+
+    def __init__(self):
+        self.calls = {}
+
+    def __getattr__(self, name):
+        if not name.startswith("fp8bw_"):
+            raise AttributeError(name)
+
+        def call(*args):
+            self.calls[name] = self.calls.get(name, 0) + 1
+        return call
+
+
+class _FakeLinear:
+    def __init__(self, kind, k, n):
+        import torch
+        self.kind, self.k, self.n = kind, k, n
+        for attr in ("qx", "sx", "qw", "sw", "qw_t", "qdy", "sdy", "qdy_t",
+                     "sdy_t", "qx_t", "sx_t", "y", "dx"):
+            setattr(self, attr, torch.zeros(1))
+
+    def ops(self, o, stream, pow2=False):
+        return [("quant_weight_block", 1e6, lambda: None),
+                ("quant_rowcol", 1e6, lambda: None),
+                ("gemm_block_scaled", 1e9, lambda: None),
+                ("gemm_vector_scaled", 1e9, lambda: None)]
+
+
+def test_next_rows_host_logic_with_stubbed_device(monkeypatch):
+    """time_next_rows end to end on the CPU: CUDA events and streams stubbed,
+    every library call a no-op; checks the rows, their units and texts."""
+    import contextlib
+    import torch
+    monkeypatch.setattr(torch.cuda, "Event", _FakeEvent)
+    monkeypatch.setattr(torch.cuda, "stream", lambda s: contextlib.nullcontext())
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a: None)
+    monkeypatch.setattr(bench, "TOKENS", 256)
+    lib = _FakeLibrary()
+    bufs = [_FakeLinear("gate_up", 128, 256), _FakeLinear("down", 256, 128)]
+    out = bench.time_next_rows(lib, bufs, None, 3, 5)
+    assert set(out) == {"wgrad_f32_accumulate", "gemm_fused_rowwise_quant",
+                        "pow2_step"}
+    assert "gate/up and down linears" in out["wgrad_f32_accumulate"]["what"]
+    assert "gate/up and down linears" in out["gemm_fused_rowwise_quant"]["what"]
+    assert ("%d-layer" % bench.LAYERS) in out["pow2_step"]["what"]
+    assert out["wgrad_f32_accumulate"]["launches"] == 5 * len(bufs)
+    assert lib.calls["fp8bw_gemm_wgrad_f32"] == 2 * (3 + 5)
+    assert lib.calls["fp8bw_gemm_fprop_quant"] == lib.calls["fp8bw_gemm_fprop"]
+    assert set(out["pow2_step"]["breakdown"]) == {
+        "quant_weight_block", "quant_rowcol", "gemm_block_scaled",
+        "gemm_vector_scaled"}
+    assert all(v["unit"] == "TFLOP/s" for k, v in out.items())
