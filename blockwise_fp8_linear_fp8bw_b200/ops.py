@@ -45,10 +45,48 @@ def _ptr(t):
     return t.data_ptr()
 
 
-def _stream(stream):
+def _stream(stream, dev=None):
+    """The raw handle of `stream`; None means the current stream of `dev`
+    (of the current device when `dev` is None). A torch stream must belong
+    to `dev`."""
     if stream is None:
-        stream = torch.cuda.current_stream()
-    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+        stream = torch.cuda.current_stream(dev)
+    if hasattr(stream, "cuda_stream"):
+        if dev is not None and stream.device != dev:
+            raise ValueError("stream is on %s, the tensors on %s"
+                             % (stream.device, dev))
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _device_of(tensors):
+    """The one CUDA device that holds every (non-None) tensor."""
+    devs = set()
+    for t in tensors:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("expected a CUDA tensor")
+        devs.add(t.device)
+    if len(devs) != 1:
+        raise ValueError("expected tensors on one CUDA device, got %s"
+                         % sorted(str(d) for d in devs))
+    return devs.pop()
+
+
+def _call(name, tensors, stream, *args):
+    """Call entry point `name` with `args` and the stream handle, on the
+    device that holds `tensors`: the library launches on the current device,
+    so a call for another device runs under a device guard."""
+    dev = _device_of(tensors)
+    handle = _stream(stream, dev)
+    fn = getattr(_lib, name)
+    if dev.index == torch.cuda.current_device():
+        status = fn(*args, handle)
+    else:
+        with torch.cuda.device(dev):
+            status = fn(*args, handle)
+    _check(status, name)
 
 
 def _expect(t, dtype, shape, name):
@@ -73,10 +111,8 @@ def fp8bw_quantize_rowwise(x, q, s, stream=None, pow2=False):
     _expect(x, torch.bfloat16, (rows, cols), "x")
     _expect(q, torch.uint8, (rows, cols), "q")
     _expect(s, torch.float32, (_cdiv(cols, 128), rows), "s")
-    name = _fn('fp8bw_quantize_rowwise', pow2)
-    _check(getattr(_lib, name)(_ptr(x), rows, cols, _ptr(q), _ptr(s),
-                               _stream(stream)),
-           name)
+    _call(_fn('fp8bw_quantize_rowwise', pow2), (x, q, s), stream,
+          _ptr(x), rows, cols, _ptr(q), _ptr(s))
 
 
 def fp8bw_quantize_colwise(x, q_t, s_t, q_row=None, s_row=None, stream=None,
@@ -88,11 +124,9 @@ def fp8bw_quantize_colwise(x, q_t, s_t, q_row=None, s_row=None, stream=None,
     if q_row is not None:
         _expect(q_row, torch.uint8, (rows, cols), "q_row")
         _expect(s_row, torch.float32, (_cdiv(cols, 128), rows), "s_row")
-    name = _fn('fp8bw_quantize_colwise', pow2)
-    _check(getattr(_lib, name)(_ptr(x), rows, cols, _ptr(q_t),
-                               _ptr(s_t), _ptr(q_row), _ptr(s_row),
-                               _stream(stream)),
-           name)
+    _call(_fn('fp8bw_quantize_colwise', pow2), (x, q_t, s_t, q_row, s_row),
+          stream, _ptr(x), rows, cols, _ptr(q_t), _ptr(s_t), _ptr(q_row),
+          _ptr(s_row))
 
 
 def fp8bw_quantize_weight_block(w, q, s, q_t=None, stream=None,
@@ -103,98 +137,92 @@ def fp8bw_quantize_weight_block(w, q, s, q_t=None, stream=None,
     _expect(s, torch.float32, (_cdiv(n, 128), _cdiv(k, 128)), "s")
     if q_t is not None:
         _expect(q_t, torch.uint8, (k, n), "q_t")
-    name = _fn('fp8bw_quantize_weight_block', pow2)
-    _check(getattr(_lib, name)(_ptr(w), n, k, _ptr(q), _ptr(s),
-                               _ptr(q_t), _stream(stream)),
-           name)
+    _call(_fn('fp8bw_quantize_weight_block', pow2), (w, q, s, q_t), stream,
+          _ptr(w), n, k, _ptr(q), _ptr(s), _ptr(q_t))
 
 
 def fp8bw_gemm_fprop(qx, sx, qw, sw, y, stream=None, pow2=False):
     m, k = qx.shape
     n = qw.shape[0]
+    _expect(qx, torch.uint8, (m, k), "qx")
     _expect(qw, torch.uint8, (n, k), "qw")
     _expect(sx, torch.float32, (_cdiv(k, 128), m), "sx")
     _expect(sw, torch.float32, (_cdiv(n, 128), _cdiv(k, 128)), "sw")
     _expect(y, torch.bfloat16, (m, n), "y")
-    name = _fn('fp8bw_gemm_fprop', pow2)
-    _check(getattr(_lib, name)(_ptr(qx), _ptr(sx), _ptr(qw), _ptr(sw), m, n,
-                               k, _ptr(y), _stream(stream)),
-           name)
+    _call(_fn('fp8bw_gemm_fprop', pow2), (qx, sx, qw, sw, y), stream,
+          _ptr(qx), _ptr(sx), _ptr(qw), _ptr(sw), m, n, k, _ptr(y))
 
 
 def fp8bw_gemm_dgrad(qdy, sdy, qw, qw_is_transposed, sw, dx, stream=None,
                      pow2=False):
     m, n = qdy.shape
     k = qw.shape[0] if qw_is_transposed else qw.shape[1]
+    _expect(qdy, torch.uint8, (m, n), "qdy")
     _expect(qw, torch.uint8, (k, n) if qw_is_transposed else (n, k), "qw")
     _expect(sdy, torch.float32, (_cdiv(n, 128), m), "sdy")
     _expect(sw, torch.float32, (_cdiv(n, 128), _cdiv(k, 128)), "sw")
     _expect(dx, torch.bfloat16, (m, k), "dx")
-    name = _fn('fp8bw_gemm_dgrad', pow2)
-    _check(getattr(_lib, name)(_ptr(qdy), _ptr(sdy), _ptr(qw),
-                               1 if qw_is_transposed else 0, _ptr(sw), m, n,
-                               k, _ptr(dx), _stream(stream)),
-           name)
+    _call(_fn('fp8bw_gemm_dgrad', pow2), (qdy, sdy, qw, sw, dx), stream,
+          _ptr(qdy), _ptr(sdy), _ptr(qw), 1 if qw_is_transposed else 0,
+          _ptr(sw), m, n, k, _ptr(dx))
 
 
 def fp8bw_gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t, dw, stream=None, pow2=False):
     n, m = qdy_t.shape
     k = qx_t.shape[0]
+    _expect(qdy_t, torch.uint8, (n, m), "qdy_t")
     _expect(qx_t, torch.uint8, (k, m), "qx_t")
     _expect(sdy_t, torch.float32, (_cdiv(m, 128), n), "sdy_t")
     _expect(sx_t, torch.float32, (_cdiv(m, 128), k), "sx_t")
     _expect(dw, torch.bfloat16, (n, k), "dw")
-    name = _fn('fp8bw_gemm_wgrad', pow2)
-    _check(getattr(_lib, name)(_ptr(qdy_t), _ptr(sdy_t), _ptr(qx_t),
-                               _ptr(sx_t), m, n, k, _ptr(dw),
-                               _stream(stream)),
-           name)
+    _call(_fn('fp8bw_gemm_wgrad', pow2), (qdy_t, sdy_t, qx_t, sx_t, dw),
+          stream, _ptr(qdy_t), _ptr(sdy_t), _ptr(qx_t), _ptr(sx_t), m, n, k,
+          _ptr(dw))
 
 
 def fp8bw_gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, dw, accumulate=False,
                          stream=None):
     n, m = qdy_t.shape
     k = qx_t.shape[0]
+    _expect(qdy_t, torch.uint8, (n, m), "qdy_t")
     _expect(qx_t, torch.uint8, (k, m), "qx_t")
     _expect(sdy_t, torch.float32, (_cdiv(m, 128), n), "sdy_t")
     _expect(sx_t, torch.float32, (_cdiv(m, 128), k), "sx_t")
     _expect(dw, torch.float32, (n, k), "dw")
-    _check(_lib.fp8bw_gemm_wgrad_f32(_ptr(qdy_t), _ptr(sdy_t), _ptr(qx_t),
-                                     _ptr(sx_t), m, n, k, _ptr(dw),
-                                     1 if accumulate else 0, _stream(stream)),
-           "fp8bw_gemm_wgrad_f32")
+    _call("fp8bw_gemm_wgrad_f32", (qdy_t, sdy_t, qx_t, sx_t, dw), stream,
+          _ptr(qdy_t), _ptr(sdy_t), _ptr(qx_t), _ptr(sx_t), m, n, k,
+          _ptr(dw), 1 if accumulate else 0)
 
 
 def fp8bw_gemm_fprop_quant(qx, sx, qw, sw, y, qy, sy, stream=None):
     m, k = qx.shape
     n = qw.shape[0]
+    _expect(qx, torch.uint8, (m, k), "qx")
     _expect(qw, torch.uint8, (n, k), "qw")
     _expect(sx, torch.float32, (_cdiv(k, 128), m), "sx")
     _expect(sw, torch.float32, (_cdiv(n, 128), _cdiv(k, 128)), "sw")
     _expect(y, torch.bfloat16, (m, n), "y")
     _expect(qy, torch.uint8, (m, n), "qy")
     _expect(sy, torch.float32, (_cdiv(n, 128), m), "sy")
-    _check(_lib.fp8bw_gemm_fprop_quant(_ptr(qx), _ptr(sx), _ptr(qw), _ptr(sw),
-                                       m, n, k, _ptr(y), _ptr(qy), _ptr(sy),
-                                       _stream(stream)),
-           "fp8bw_gemm_fprop_quant")
+    _call("fp8bw_gemm_fprop_quant", (qx, sx, qw, sw, y, qy, sy), stream,
+          _ptr(qx), _ptr(sx), _ptr(qw), _ptr(sw), m, n, k, _ptr(y), _ptr(qy),
+          _ptr(sy))
 
 
 def fp8bw_gemm_dgrad_quant(qdy, sdy, qw, qw_is_transposed, sw, dx, qdx, sdx,
                            stream=None):
     m, n = qdy.shape
     k = qw.shape[0] if qw_is_transposed else qw.shape[1]
+    _expect(qdy, torch.uint8, (m, n), "qdy")
     _expect(qw, torch.uint8, (k, n) if qw_is_transposed else (n, k), "qw")
     _expect(sdy, torch.float32, (_cdiv(n, 128), m), "sdy")
     _expect(sw, torch.float32, (_cdiv(n, 128), _cdiv(k, 128)), "sw")
     _expect(dx, torch.bfloat16, (m, k), "dx")
     _expect(qdx, torch.uint8, (m, k), "qdx")
     _expect(sdx, torch.float32, (_cdiv(k, 128), m), "sdx")
-    _check(_lib.fp8bw_gemm_dgrad_quant(_ptr(qdy), _ptr(sdy), _ptr(qw),
-                                       1 if qw_is_transposed else 0, _ptr(sw),
-                                       m, n, k, _ptr(dx), _ptr(qdx), _ptr(sdx),
-                                       _stream(stream)),
-           "fp8bw_gemm_dgrad_quant")
+    _call("fp8bw_gemm_dgrad_quant", (qdy, sdy, qw, sw, dx, qdx, sdx), stream,
+          _ptr(qdy), _ptr(sdy), _ptr(qw), 1 if qw_is_transposed else 0,
+          _ptr(sw), m, n, k, _ptr(dx), _ptr(qdx), _ptr(sdx))
 
 
 def fp8bw_selftest_wait_timeout(limit_ns, stream=None):
