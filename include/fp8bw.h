@@ -25,6 +25,9 @@
  *   - All data pointers are DEVICE pointers owned by the caller. The library
  *     never allocates, frees or keeps them. Outputs must not alias inputs. A
  *     pointer may be NULL only when its buffer holds no element.
+ *   - A call runs on the calling thread's current CUDA device: its pointers
+ *     and `stream` must belong to that device (the library cannot tell which
+ *     device a pointer belongs to; memory of another GPU is not supported).
  *   - bf16 tensors are passed as uint16_t bit patterns. FP8 codes are uint8_t
  *     OCP E4M3 codes. Scales are fp32.
  *   - Matrices are dense row-major (leading dimension = row length).
