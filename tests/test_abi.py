@@ -217,3 +217,24 @@ def test_header_builds_a_plain_client(lib, tmp_path, compiler, std):
     null_msg, ok_msg = rest.split("|")
     assert null_msg == lib.fp8bw_status_string(E_NULL).decode()
     assert ok_msg == lib.fp8bw_status_string(OK).decode()
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """No CPU fallback: without libfp8bw.so (and nothing to build it from) the
+    loader raises instead of returning anything callable."""
+    from blockwise_fp8_linear_fp8bw_b200 import build as _build
+    monkeypatch.setattr(_native, "_lib", None)
+    monkeypatch.setattr(_native, "LIB_PATH", str(tmp_path / "libfp8bw.so"))
+    monkeypatch.setattr(_build, "needs_build", lambda: False)
+    with pytest.raises(ImportError, match="missing"):
+        _native.load()
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    """No CPU fallback in the binding either: CPU tensors are refused before
+    the library is reached, and nothing is computed."""
+    import torch
+    from blockwise_fp8_linear_fp8bw_b200 import ops
+    x = torch.zeros((128, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        ops.quantize_rowwise(x)
