@@ -1,4 +1,7 @@
-"""Shared test helpers: tensor conversion, parity tolerance, sample points."""
+"""Shared test helpers: tensor conversion, parity tolerance, sample points,
+the hand-worked golden groups."""
+import os
+
 import numpy as np
 
 import oracle
@@ -101,3 +104,23 @@ __all__ = ["bf16_np_to_torch", "torch_bf16_to_np", "bf16_bits_to_f64",
            "ulp_bf16", "gemm_tolerance", "assert_gemm_close", "ulp_f32",
            "assert_gemm_close_f32",
            "sample_points", "scale_bits", "oracle"]
+
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def hand_groups(fname="quant_group_hand.txt"):
+    """Rows of a hand-worked group file: (name, listed values, fill value,
+    expected codes of the listed values, expected scale bits)."""
+    rows = []
+    with open(os.path.join(GOLDEN, fname)) as fh:
+        for line in fh:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            name, vals, fill, codes, sbits = [p.strip() for p in line.split("|")]
+            ev = lambda e: float(eval(e, {"__builtins__": {}}))  # noqa: E731
+            rows.append((name, [ev(v) for v in vals.split(",")], ev(fill),
+                         [int(c, 16) for c in codes.split(",")],
+                         int(sbits, 16)))
+    return rows

@@ -8,7 +8,7 @@ import pytest
 
 import oracle
 import synthetic as S
-from helpers import bf16_np_to_torch, scale_bits
+from helpers import bf16_np_to_torch, hand_groups, scale_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -89,6 +89,42 @@ def test_special_groups():
     _check_rowwise(x)
     _check_colwise(x, True)
     _check_weight(x)
+
+
+@pytest.mark.parametrize("pow2,fname", [(False, "quant_group_hand.txt"),
+                                         (True, "quant_pow2_hand.txt")])
+def test_hand_worked_groups(pow2, fname):
+    """The hand-worked golden groups (values, codes and scale bits derived by
+    hand, tests/golden/) through every quantiser: each group as a row-wise
+    1x128 group, as a column-wise 128x1 group and as the only non-zero row of
+    a 128x128 weight block (whose amax is then the group's). The file's
+    r2_* groups sit on E4M3 midpoints where multiplying by fl32(448/amax) and
+    dividing by fl32(amax/448) give different codes."""
+    ops = _ops()
+    groups = hand_groups(fname)
+    n = len(groups)
+    f = np.zeros((128 * n, 128), np.float32)
+    for i, (_name, vals, fill, _codes, _sbits) in enumerate(groups):
+        f[128 * i + 3, :] = fill
+        f[128 * i + 3, :len(vals)] = vals
+    x = (f.view(np.uint32) >> 16).astype(np.uint16)
+    assert np.array_equal((x.astype(np.uint32) << 16).view(np.float32), f)
+    xt = np.ascontiguousarray(x.T)                     # groups as columns
+    q, s = ops.quantize_rowwise(bf16_np_to_torch(x), pow2=pow2)
+    q_t, s_t = ops.quantize_colwise(bf16_np_to_torch(xt), pow2=pow2)
+    qb, sb, _ = ops.quantize_weight_block(bf16_np_to_torch(x), pow2=pow2)
+    ops.fp8bw_check_device_error()
+    q, s = q.cpu().numpy(), scale_bits(s.cpu().numpy())
+    q_t, s_t = q_t.cpu().numpy(), scale_bits(s_t.cpu().numpy())
+    qb, sb = qb.cpu().numpy(), scale_bits(sb.cpu().numpy())
+    for i, (name, vals, _fill, codes, sbits) in enumerate(groups):
+        r = 128 * i + 3
+        assert q[r, :len(codes)].tolist() == codes, name
+        assert s[0, r] == sbits, name
+        assert q_t[r, :len(codes)].tolist() == codes, name     # q_t[col][tok]
+        assert s_t[0, r] == sbits, name
+        assert qb[r, :len(codes)].tolist() == codes, name
+        assert sb[i, 0] == sbits, name
 
 
 def test_empty_is_a_noop():

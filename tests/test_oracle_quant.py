@@ -6,15 +6,12 @@ Reading of the pages (Puro-2B arxiv-wiki summary, Approach item (4): E4M3,
 activation 1-D groups of 128, weight 128x128 blocks): qscale = fl(448/amax),
 s = fl(amax/448), all-zero groups get qscale = s = 1.
 """
-import os
-
 import numpy as np
 import pytest
 
 import oracle
 import synthetic as S
-
-GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+from helpers import hand_groups
 
 
 def bf16_bits(vals):
@@ -28,22 +25,7 @@ def f32_of(b):
     return (np.asarray(b, np.uint16).astype(np.uint32) << 16).view(np.float32)
 
 
-def _hand_groups(fname="quant_group_hand.txt"):
-    rows = []
-    with open(os.path.join(GOLDEN, fname)) as fh:
-        for line in fh:
-            line = line.strip()
-            if not line or line.startswith("#"):
-                continue
-            name, vals, fill, codes, sbits = [p.strip() for p in line.split("|")]
-            ev = lambda e: float(eval(e, {"__builtins__": {}}))
-            rows.append((name, [ev(v) for v in vals.split(",")], ev(fill),
-                         [int(c, 16) for c in codes.split(",")],
-                         int(sbits, 16)))
-    return rows
-
-
-@pytest.mark.parametrize("name,vals,fill,codes,sbits", _hand_groups())
+@pytest.mark.parametrize("name,vals,fill,codes,sbits", hand_groups())
 def test_hand_worked_group(name, vals, fill, codes, sbits):
     g = np.full(128, fill, dtype=np.float32)
     g[: len(vals)] = vals
@@ -164,7 +146,7 @@ def test_roundtrip_bound_rowwise_colwise_weight():
 # E the smallest integer with 448 * 2^E >= amax, clamped to [-127, 127].
 
 @pytest.mark.parametrize("name,vals,fill,codes,sbits",
-                         _hand_groups("quant_pow2_hand.txt"))
+                         hand_groups("quant_pow2_hand.txt"))
 def test_pow2_hand_worked_group(name, vals, fill, codes, sbits):
     g = np.full(128, fill, dtype=np.float32)
     g[: len(vals)] = vals
