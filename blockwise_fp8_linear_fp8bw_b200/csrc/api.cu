@@ -27,11 +27,10 @@ namespace fp8bw {
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-
 struct DeviceInfo {
   int checked = 0;      // 0 = unknown, 1 = sm_100, -1 = other
   int sm_count = 0;
+  int ordinal = 0;      // CUDA device ordinal
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -55,6 +54,7 @@ int current_device_info(DeviceInfo* out) {
       return FP8BW_ERR_DEVICE;
     d.checked = (major == 10 && minor == 0) ? 1 : -1;
     d.sm_count = sms;
+    d.ordinal = dev;
   }
   if (d.checked != 1) return FP8BW_ERR_DEVICE;
   *out = d;
@@ -166,6 +166,24 @@ int encode_f32_out(CUtensorMap* map, void* base, uint64_t cols, uint64_t rows) {
 }
 
 // --------------------------------------------------------------- GEMM launch
+// How many clusters of two CTAs of `kernel` fit on the device at once.
+int max_active_clusters(const void* kernel, int threads, int smem_bytes, int sm_count, int* out) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * sm_count, 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.dynamicSmemBytes = smem_bytes;
+  cudaLaunchAttribute attr_cl;
+  attr_cl.id = cudaLaunchAttributeClusterDimension;
+  attr_cl.val.clusterDim.x = 2;
+  attr_cl.val.clusterDim.y = 1;
+  attr_cl.val.clusterDim.z = 1;
+  cfg.attrs = &attr_cl;
+  cfg.numAttrs = 1;
+  if (cudaOccupancyMaxActiveClusters(out, kernel, &cfg) != cudaSuccess || *out < 1)
+    return FP8BW_ERR_LAUNCH;
+  return FP8BW_OK;
+}
+
 struct GemmProblem {
   const uint8_t* a;  // [mo][kc]
   const uint8_t* b;  // K-major: [no][kc]; MN-major: [kc][no]
@@ -187,38 +205,21 @@ template <int BN, bool VEC_B, bool B_MN, int OUT = gemm::kOutBf16>
 int launch_gemm_pair(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t stream) {
   using L = gemm::PairLayout<BN, VEC_B>;
   auto kernel = gemm::blockwise_gemm_pair_kernel<BN, VEC_B, B_MN, OUT>;
-  static std::once_flag once;
-  static int prep_status = FP8BW_OK;
-  static int max_clusters = 0;
-  std::call_once(once, [&]() {
+  static DevicePrep prep;
+  int max_clusters = 0;
+  const int prep_status = prepare_for_device(prep, dev.ordinal, &max_clusters, [&](int* mc) {
     cudaFuncAttributes attr;
     // With BN = 256 the kernel redistributes registers with setmaxnreg, which
     // draws on exactly the launch allocation: refuse to launch if that
     // allocation is smaller than the split assumes.
     if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess ||
-        (BN == 256 && attr.numRegs < gemm::kLaunchRegs)) {
-      prep_status = FP8BW_ERR_LAUNCH;
-      return;
-    }
+        (BN == 256 && attr.numRegs < gemm::kLaunchRegs))
+      return static_cast<int>(FP8BW_ERR_LAUNCH);
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) !=
-        cudaSuccess) {
-      prep_status = FP8BW_ERR_LAUNCH;
-      return;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * dev.sm_count, 1, 1);
-    cfg.blockDim = dim3(gemm::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = L::kAlloc;
-    cudaLaunchAttribute attr_cl;
-    attr_cl.id = cudaLaunchAttributeClusterDimension;
-    attr_cl.val.clusterDim.x = 2;
-    attr_cl.val.clusterDim.y = 1;
-    attr_cl.val.clusterDim.z = 1;
-    cfg.attrs = &attr_cl;
-    cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&max_clusters, kernel, &cfg) != cudaSuccess ||
-        max_clusters < 1)
-      prep_status = FP8BW_ERR_LAUNCH;
+        cudaSuccess)
+      return static_cast<int>(FP8BW_ERR_LAUNCH);
+    return max_active_clusters(reinterpret_cast<const void*>(kernel), gemm::kThreads, L::kAlloc,
+                               dev.sm_count, mc);
   });
   if (prep_status != FP8BW_OK) return prep_status;
 
@@ -265,29 +266,14 @@ template <bool VEC_B, bool B_MN>
 int launch_gemm_pow2(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t stream) {
   using L = gemm_pow2::Layout;
   auto kernel = gemm_pow2::blockwise_gemm_pow2_kernel<VEC_B, B_MN>;
-  static std::once_flag once;
-  static int prep_status = FP8BW_OK;
-  static int max_clusters = 0;
-  std::call_once(once, [&]() {
+  static DevicePrep prep;
+  int max_clusters = 0;
+  const int prep_status = prepare_for_device(prep, dev.ordinal, &max_clusters, [&](int* mc) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) !=
-        cudaSuccess) {
-      prep_status = FP8BW_ERR_LAUNCH;
-      return;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * dev.sm_count, 1, 1);
-    cfg.blockDim = dim3(gemm_pow2::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = L::kAlloc;
-    cudaLaunchAttribute attr_cl;
-    attr_cl.id = cudaLaunchAttributeClusterDimension;
-    attr_cl.val.clusterDim.x = 2;
-    attr_cl.val.clusterDim.y = 1;
-    attr_cl.val.clusterDim.z = 1;
-    cfg.attrs = &attr_cl;
-    cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&max_clusters, kernel, &cfg) != cudaSuccess ||
-        max_clusters < 1)
-      prep_status = FP8BW_ERR_LAUNCH;
+        cudaSuccess)
+      return static_cast<int>(FP8BW_ERR_LAUNCH);
+    return max_active_clusters(reinterpret_cast<const void*>(kernel), gemm_pow2::kThreads,
+                               L::kAlloc, dev.sm_count, mc);
   });
   if (prep_status != FP8BW_OK) return prep_status;
 
@@ -352,7 +338,7 @@ int run_gemm(const GemmProblem& p, cudaStream_t stream) {
     if (p.out_mode != gemm::kOutBf16Q) return FP8BW_OK;
     // ... and its row-wise quantisation is that of a zero matrix
     return launch_quantize(kModeRow, false, static_cast<const uint16_t*>(p.out), p.mo, p.no,
-                           p.q_out, p.s_out, nullptr, nullptr, nullptr, dev.sm_count, stream);
+                           p.q_out, p.s_out, nullptr, nullptr, nullptr, dev.ordinal, dev.sm_count, stream);
   }
   if (cdiv(p.mo, 256) * cdiv(p.no, 256) > (int64_t(1) << 30)) return FP8BW_ERR_SHAPE;
   if (p.pow2) {
@@ -420,7 +406,7 @@ int quantize_rowwise(bool pow2, const uint16_t* x, int64_t rows, int64_t cols, u
   int st = current_device_info(&dev);
   if (st != FP8BW_OK) return st;
   if (rows == 0 || cols == 0) return FP8BW_OK;
-  return launch_quantize(kModeRow, pow2, x, rows, cols, q, s, nullptr, nullptr, nullptr, dev.sm_count,
+  return launch_quantize(kModeRow, pow2, x, rows, cols, q, s, nullptr, nullptr, nullptr, dev.ordinal, dev.sm_count,
                          static_cast<cudaStream_t>(stream));
 }
 
@@ -446,7 +432,7 @@ int quantize_colwise(bool pow2, const uint16_t* x, int64_t rows, int64_t cols, u
   if (st != FP8BW_OK) return st;
   if (rows == 0 || cols == 0) return FP8BW_OK;
   const int mode = q_row ? kModeRowCol : kModeCol;
-  return launch_quantize(mode, pow2, x, rows, cols, q_row, s_row, q_t, s_t, nullptr, dev.sm_count,
+  return launch_quantize(mode, pow2, x, rows, cols, q_row, s_row, q_t, s_t, nullptr, dev.ordinal, dev.sm_count,
                          static_cast<cudaStream_t>(stream));
 }
 
@@ -466,7 +452,7 @@ int quantize_weight_block(bool pow2, const uint16_t* w, int64_t n, int64_t k, ui
   int st = current_device_info(&dev);
   if (st != FP8BW_OK) return st;
   if (n == 0 || k == 0) return FP8BW_OK;
-  return launch_quantize(kModeBlock, pow2, w, n, k, q, nullptr, q_t, nullptr, s, dev.sm_count,
+  return launch_quantize(kModeBlock, pow2, w, n, k, q, nullptr, q_t, nullptr, s, dev.ordinal, dev.sm_count,
                          static_cast<cudaStream_t>(stream));
 }
 

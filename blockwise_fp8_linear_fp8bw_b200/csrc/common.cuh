@@ -3,7 +3,9 @@
 // tcgen05 (5th-generation tensor core, TMEM) instructions as inline PTX.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
+#include <mutex>
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
@@ -11,6 +13,43 @@
 #include "../../include/fp8bw.h"
 
 namespace fp8bw {
+
+// ---------------------------------------------------------------------------
+// Host: one-time set-up of a kernel per device. Function attributes (the
+// dynamic shared-memory size) and occupancy answers belong to a device's
+// context, so every device the library is called on gets its own set-up.
+// ---------------------------------------------------------------------------
+constexpr int kMaxDevices = 64;
+
+struct DevicePrep {
+  std::atomic<int> done[kMaxDevices];   // static storage: starts at 0
+  int status[kMaxDevices];
+  int value[kMaxDevices];
+};
+
+inline std::mutex& device_prep_mutex() {
+  static std::mutex m;
+  return m;
+}
+
+// The first call for device `dev` runs fn(&value) (an fp8bw status); every
+// call for `dev` returns that status and stores that value in *value. The
+// device must be current on the calling thread.
+template <typename Fn>
+int prepare_for_device(DevicePrep& p, int dev, int* value, Fn&& fn) {
+  if (dev < 0 || dev >= kMaxDevices) return FP8BW_ERR_DEVICE;
+  if (!p.done[dev].load(std::memory_order_acquire)) {
+    std::lock_guard<std::mutex> lock(device_prep_mutex());
+    if (!p.done[dev].load(std::memory_order_relaxed)) {
+      int v = 0;
+      p.status[dev] = fn(&v);
+      p.value[dev] = v;
+      p.done[dev].store(1, std::memory_order_release);
+    }
+  }
+  *value = p.value[dev];
+  return p.status[dev];
+}
 
 // ---------------------------------------------------------------------------
 // Device error record. A kernel whose bounded wait expires ORs a bit in here

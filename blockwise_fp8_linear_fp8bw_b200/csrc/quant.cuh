@@ -32,8 +32,6 @@
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
-#include <mutex>
-
 #include "common.cuh"
 
 namespace fp8bw {
@@ -344,7 +342,7 @@ int encode_bf16_in(CUtensorMap* map, const void* base, uint64_t cols, uint64_t r
 // Launchers (shapes and pointers already validated by the C ABI layer).
 int launch_quantize(int mode, bool pow2, const uint16_t* x, int64_t rows, int64_t cols,
                     uint8_t* q_row, float* s_row, uint8_t* q_col, float* s_col, float* s_block,
-                    int sm_count, cudaStream_t stream) {
+                    int device, int sm_count, cudaStream_t stream) {
   QuantArgs a{rows, cols, static_cast<int>((rows + kQTile - 1) / kQTile),
               static_cast<int>((cols + kQTile - 1) / kQTile), q_row, s_row, q_col, s_col, s_block};
   CUtensorMap tm;
@@ -358,15 +356,16 @@ int launch_quantize(int mode, bool pow2, const uint16_t* x, int64_t rows, int64_
       quant_tile_kernel<kModeRowCol, false>, quant_tile_kernel<kModeBlock, false>,
       quant_tile_kernel<kModeRow, true>,     quant_tile_kernel<kModeCol, true>,
       quant_tile_kernel<kModeRowCol, true>,  quant_tile_kernel<kModeBlock, true>};
-  static std::once_flag once;
-  static int prep = FP8BW_OK;
-  std::call_once(once, [&]() {
+  static DevicePrep prep;
+  int unused = 0;
+  const int pst = prepare_for_device(prep, device, &unused, [&](int*) {
     for (Kernel k : kernels)
       if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                QuantSmem::kAlloc) != cudaSuccess)
-        prep = FP8BW_ERR_LAUNCH;
+        return static_cast<int>(FP8BW_ERR_LAUNCH);
+    return static_cast<int>(FP8BW_OK);
   });
-  if (prep != FP8BW_OK) return prep;
+  if (pst != FP8BW_OK) return pst;
   const Kernel kernel = kernels[(mode >= 0 && mode < 4 ? mode : kModeBlock) + (pow2 ? 4 : 0)];
   kernel<<<grid, kQThreads, QuantSmem::kAlloc, stream>>>(tm, a);
   return cudaGetLastError() == cudaSuccess ? FP8BW_OK : FP8BW_ERR_LAUNCH;

@@ -41,12 +41,13 @@ def wgrad_all_reduce(qdy_t, sdy_t, qx_t, sx_t, group=None, stream=None):
     (its token shard, see token_shard). Returns the fp32 [n, k] sum over the
     process group of the replicas' local dW; every replica must call this
     with the same n and k. The all-reduce is ordered after the local GEMM on
-    `stream` (default: the current stream)."""
+    `stream` (default: the current stream of the device that holds the
+    shards)."""
     import torch.distributed as dist
 
     from . import ops
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(qdy_t.device)
     dw = ops.gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, stream=stream)
     if dist.is_available() and dist.is_initialized():
         with torch.cuda.stream(stream):

@@ -225,14 +225,36 @@ def fp8bw_gemm_dgrad_quant(qdy, sdy, qw, qw_is_transposed, sw, dx, qdx, sdx,
           _ptr(sw), m, n, k, _ptr(dx), _ptr(qdx), _ptr(sdx))
 
 
-def fp8bw_selftest_wait_timeout(limit_ns, stream=None):
-    _check(_lib.fp8bw_selftest_wait_timeout(int(limit_ns), _stream(stream)),
-           "fp8bw_selftest_wait_timeout")
+def _device_call(name, stream, device, *args):
+    """Call a device-wide entry point (no tensor arguments) for one device:
+    `device` if given, else the device of a torch `stream`, else the current
+    device. The library works on the current device, so another device's
+    call runs under a device guard."""
+    if device is None and hasattr(stream, "device"):
+        device = stream.device
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None \
+        else torch.device(device)
+    if dev.type != "cuda" or dev.index is None:
+        raise ValueError("expected a CUDA device with an index, got %s" % dev)
+    handle = _stream(stream, dev)
+    fn = getattr(_lib, name)
+    if dev.index == torch.cuda.current_device():
+        status = fn(*args, handle)
+    else:
+        with torch.cuda.device(dev):
+            status = fn(*args, handle)
+    _check(status, name)
 
 
-def fp8bw_check_device_error(stream=None):
-    _check(_lib.fp8bw_check_device_error(_stream(stream)),
-           "fp8bw_check_device_error")
+def fp8bw_selftest_wait_timeout(limit_ns, stream=None, device=None):
+    _device_call("fp8bw_selftest_wait_timeout", stream, device, int(limit_ns))
+
+
+def fp8bw_check_device_error(stream=None, device=None):
+    """Synchronise `stream` and raise Fp8bwError if a kernel of the library on
+    that device (`device`, else the stream's, else the current one) recorded
+    an expired wait or a bad power-of-two scale since the last check."""
+    _device_call("fp8bw_check_device_error", stream, device)
 
 
 # ----------------------------------------------------------- allocating helpers

@@ -148,3 +148,40 @@ def test_optional_outputs_may_be_absent(lib):
     assert name == "fp8bw_quantize_colwise" and dev == 1
     assert args == (x.data_ptr(), 256, 512, q_t.data_ptr(), s_t.data_ptr(),
                     None, None, 1001)
+
+
+def test_device_error_check_goes_to_the_stream_or_given_device(lib):
+    # the error record is per device: a check for device 1 must run with
+    # device 1 current and device 1's stream, whatever torch's current one is
+    ops.fp8bw_check_device_error(_Stream(1, 66))
+    name, args, dev = lib.calls[-1]
+    assert name == "fp8bw_check_device_error" and dev == 1 and args == (66,)
+    ops.fp8bw_check_device_error(device=1)
+    assert lib.calls[-1] == ("fp8bw_check_device_error", (1001,), 1)
+    ops.fp8bw_check_device_error()
+    assert lib.calls[-1] == ("fp8bw_check_device_error", (1000,), 0)
+    with pytest.raises(ValueError, match="stream"):
+        ops.fp8bw_check_device_error(_Stream(0, 5), device=1)
+    ops.fp8bw_selftest_wait_timeout(1000, device=1)
+    assert lib.calls[-1] == ("fp8bw_selftest_wait_timeout", (1000, 1001), 1)
+    assert _State.device == 0
+
+
+def test_data_parallel_default_stream_is_the_shards_device(lib, monkeypatch):
+    from blockwise_fp8_linear_fp8bw_b200 import data_parallel as dp
+    n, k, m = 256, 384, 512
+    u8, f32 = torch.uint8, torch.float32
+    qdy_t, sdy_t = _Tensor((n, m), u8, 1), _Tensor((m // 128, n), f32, 1)
+    qx_t, sx_t = _Tensor((k, m), u8, 1), _Tensor((m // 128, k), f32, 1)
+    made = []
+
+    def fake_empty(shape, dtype, device):
+        t = _Tensor(shape, dtype, torch.device(device).index)
+        made.append(t)
+        return t
+    monkeypatch.setattr(torch, "empty", fake_empty)
+    monkeypatch.setattr(torch.distributed, "is_initialized", lambda: False)
+    dw = dp.wgrad_all_reduce(qdy_t, sdy_t, qx_t, sx_t)
+    name, args, dev = lib.calls[-1]
+    assert name == "fp8bw_gemm_wgrad_f32" and dev == 1
+    assert args[-1] == 1001 and dw is made[-1]
