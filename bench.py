@@ -84,7 +84,7 @@ def ncu_traffic(kernel):
     return NCU_TRAFFIC_PER_LAUNCH.get(kernel)
 
 
-def parse_args():
+def parse_args(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=20)
@@ -98,7 +98,7 @@ def parse_args():
                    help="layers per step (profiling runs use fewer)")
     p.add_argument("--linears", default="qkv,o,gate_up,down",
                    help="comma list of the linears in a layer")
-    args = p.parse_args()
+    args = p.parse_args(argv)
     global LAYERS, KINDS
     LAYERS = args.layers
     KINDS = tuple(args.linears.split(","))
@@ -119,6 +119,55 @@ def dist_env():
     return (int(os.environ.get("WORLD_SIZE", "1")),
             int(os.environ.get("RANK", "0")),
             int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def free_port():
+    import socket
+    with socket.socket() as sock:
+        sock.bind(("127.0.0.1", 0))
+        return sock.getsockname()[1]
+
+
+def launch_ranks(n, argv, script=None, timeout_s=3600):
+    """Start `n` ranks of `script` (this file by default) with the arguments
+    `argv`, one process per GPU on this node, under torch.distributed.run
+    with a 127.0.0.1 rendezvous; returns the launcher's exit status. The
+    launcher runs in its own process group, ended as a whole if it outlives
+    `timeout_s`."""
+    import signal
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           "--nproc-per-node", str(n), "--master-addr", "127.0.0.1",
+           "--master-port", str(free_port()),
+           script or os.path.abspath(__file__)] + list(argv)
+    proc = subprocess.Popen(cmd, start_new_session=True)
+    try:
+        return proc.wait(timeout=timeout_s)
+    except subprocess.TimeoutExpired:
+        os.killpg(proc.pid, signal.SIGTERM)
+        try:
+            proc.wait(timeout=60)
+        except subprocess.TimeoutExpired:
+            os.killpg(proc.pid, signal.SIGKILL)
+            proc.wait()
+        return 124
+
+
+def check_launch(gpus):
+    """None when this process should run the benchmark itself; else the exit
+    status to return: `--gpus N` (N > 1) outside a torchrun launch starts N
+    ranks (launch_ranks) and reports their status; inside one, WORLD_SIZE
+    must equal N."""
+    if "WORLD_SIZE" not in os.environ:
+        if gpus > 1:
+            return launch_ranks(gpus, sys.argv[1:])
+        return None
+    world = int(os.environ["WORLD_SIZE"])
+    if world != gpus:
+        sys.stderr.write("bench.py: --gpus %d but WORLD_SIZE=%d (torchrun "
+                         "--nproc-per-node must equal --gpus)\n"
+                         % (gpus, world))
+        return 2
+    return None
 
 
 def max_over_ranks(value, world, device):
@@ -205,7 +254,7 @@ class OracleSample:
 
 
 def run_reference(args):
-    _, rank, _ = dist_env()
+    world, rank, _ = dist_env()
     if rank != 0:          # the CPU oracle runs once, on rank 0
         return 0
     sample = OracleSample(tokens=64)
@@ -221,7 +270,7 @@ def run_reference(args):
         "metric": METRIC,
         "value": value,
         "unit": "TFLOP/s",
-        "n_gpus": args.gpus,
+        "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": dt * 1e3,
@@ -535,18 +584,17 @@ def gpu_uuid(torch, dev):
         return str(dev)
 
 
-def run_gpu(args):
+def measure_replica(args, world, local):
+    """Everything one rank (one GPU) measures: the timed steps, the
+    per-kernel events, the rows beyond the step and the end-to-end step.
+    Every collective here (barriers, the max over ranks) is taken by every
+    rank in the same order. Returns the values the JSON line is made of; the
+    step and e2e times are already the max over ranks."""
     import torch
     import torch.distributed as dist
 
-    world, rank, local = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", device_id=dev,
-                                timeout=datetime.timedelta(seconds=300))
-
     from blockwise_fp8_linear_fp8bw_b200 import ops as o
 
     stream = torch.cuda.Stream(device=dev)
@@ -712,12 +760,45 @@ def run_gpu(args):
                          "on a copy stream while the previous layer computes; "
                          "dW downloaded on another stream"}
 
+    return {"ms": ms, "flops": flops, "per_kind": per_kind,
+            "next_rows": next_rows, "clocks": clk, "e2e": e2e,
+            "launches_per_step": len(step_ops)}
+
+
+def run_gpu(args, measure=measure_replica):
+    """One rank of the GPU arm: joins the process group (NCCL, one process
+    per GPU) when there are several ranks, runs `measure`, and on rank 0
+    prints the JSON line."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    world, rank, local = dist_env()
     if world > 1:
-        dist.barrier(device_ids=[local])
-        dist.destroy_process_group()
+        kw = {}
+        backend = "gloo"
+        if torch.cuda.is_available():
+            backend = "nccl"
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300),
+                                **kw)
+    try:
+        res = measure(args, world, local)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
     if rank != 0:
         return 0
+    line = result_line(args, world, res)
+    print(json.dumps(line))
+    return 0
 
+
+def result_line(args, world, res):
+    """The JSON line of the GPU arm from what measure_replica returned."""
+    ms, flops, per_kind = res["ms"], res["flops"], res["per_kind"]
+    next_rows, clk, e2e = res["next_rows"], res["clocks"], res["e2e"]
     peaks = load_peaks()
     fp8_sustained = peaks["bf16_tflops_sustained"] * FP8_OVER_BF16
     breakdown = {}
@@ -795,7 +876,7 @@ def run_gpu(args):
                    "per_launch_events": "CUDA events around every launch of "
                                         "the last timed step",
                    "parallelism": "replicas" if world > 1 else "single"},
-        "gpu_launches": len(step_ops) * args.steps,
+        "gpu_launches": res["launches_per_step"] * args.steps,
         "roofline": roofline,
         "breakdown": breakdown,
         "next_rows": next_rows,
@@ -806,15 +887,17 @@ def run_gpu(args):
                   "fp8_tflops_sustained": fp8_sustained,
                   "source": peaks["source"]},
     }
-    print(json.dumps(line))
-    return 0
+    return line
 
 
-def main():
-    args = parse_args()
+def main(argv=None, measure=measure_replica):
+    args = parse_args(argv)
+    status = check_launch(args.gpus)
+    if status is not None:
+        return status
     if args.impl == "reference":
         return run_reference(args)
-    return run_gpu(args)
+    return run_gpu(args, measure)
 
 
 if __name__ == "__main__":
