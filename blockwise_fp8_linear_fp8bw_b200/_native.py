@@ -34,6 +34,8 @@ SIGNATURES = {
     "fp8bw_gemm_dgrad_pow2": ([_P, _P, _P, _INT, _P, _I64, _I64, _I64, _P,
                                _P], _INT),
     "fp8bw_gemm_wgrad_pow2": ([_P, _P, _P, _P, _I64, _I64, _I64, _P, _P], _INT),
+    "fp8bw_gemm_wgrad_f32_pow2": ([_P, _P, _P, _P, _I64, _I64, _I64, _P, _INT,
+                                   _P], _INT),
     "fp8bw_selftest_wait_timeout": ([_I64, _P], _INT),
     "fp8bw_check_device_error": ([_P], _INT),
     "fp8bw_status_string": ([_INT], ctypes.c_char_p),

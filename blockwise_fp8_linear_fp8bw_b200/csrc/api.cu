@@ -194,14 +194,14 @@ struct GemmProblem {
   const float* sb;
   int64_t sbj, sbc;
   void* out;         // [mo][no]: bf16 (kOutBf16) or fp32
-  int out_mode;      // gemm::kOutBf16 / kOutF32 / kOutF32Add
+  int out_mode;      // kOutBf16 / kOutF32 / kOutF32Add
   bool pow2;         // power-of-two scales on the hardware block-scaled MMA
   uint8_t* q_out;    // kOutBf16Q: row-wise codes of the bf16 output [mo][no]
   float* s_out;      // kOutBf16Q: their scales [ceil(no/128)][mo]
 };
 
 // CTA-pair kernel: 256 x 256 output tiles on clusters of two CTAs.
-template <int BN, bool VEC_B, bool B_MN, int OUT = gemm::kOutBf16>
+template <int BN, bool VEC_B, bool B_MN, int OUT = kOutBf16>
 int launch_gemm_pair(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t stream) {
   using L = gemm::PairLayout<BN, VEC_B>;
   auto kernel = gemm::blockwise_gemm_pair_kernel<BN, VEC_B, B_MN, OUT>;
@@ -233,7 +233,7 @@ int launch_gemm_pair(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t s
     st = encode_u8_2d(&tm_b, p.b, static_cast<uint64_t>(p.kc), static_cast<uint64_t>(p.no),
                       BN / 2);
   if (st != FP8BW_OK) return st;
-  if (gemm::out_is_bf16(OUT))
+  if (out_is_bf16(OUT))
     st = encode_bf16_out(&tm_out, p.out, static_cast<uint64_t>(p.no),
                          static_cast<uint64_t>(p.mo));
   else
@@ -262,10 +262,10 @@ int launch_gemm_pair(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t s
 }
 
 // Power-of-two-scale kernel (hardware block scaling), same problem description.
-template <bool VEC_B, bool B_MN>
+template <bool VEC_B, bool B_MN, int OUT = kOutBf16>
 int launch_gemm_pow2(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t stream) {
   using L = gemm_pow2::Layout;
-  auto kernel = gemm_pow2::blockwise_gemm_pow2_kernel<VEC_B, B_MN>;
+  auto kernel = gemm_pow2::blockwise_gemm_pow2_kernel<VEC_B, B_MN, OUT>;
   static DevicePrep prep;
   int max_clusters = 0;
   const int prep_status = prepare_for_device(prep, dev.ordinal, &max_clusters, [&](int* mc) {
@@ -287,7 +287,10 @@ int launch_gemm_pow2(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t s
     st = encode_u8_2d(&tm_b, p.b, static_cast<uint64_t>(p.kc), static_cast<uint64_t>(p.no),
                       gemm_pow2::BN / 2);
   if (st != FP8BW_OK) return st;
-  st = encode_bf16_out(&tm_out, p.out, static_cast<uint64_t>(p.no), static_cast<uint64_t>(p.mo));
+  if (out_is_bf16(OUT))
+    st = encode_bf16_out(&tm_out, p.out, static_cast<uint64_t>(p.no), static_cast<uint64_t>(p.mo));
+  else
+    st = encode_f32_out(&tm_out, p.out, static_cast<uint64_t>(p.no), static_cast<uint64_t>(p.mo));
   if (st != FP8BW_OK) return st;
 
   gemm_pow2::Args g;
@@ -330,32 +333,36 @@ int run_gemm(const GemmProblem& p, cudaStream_t stream) {
   if (p.mo == 0 || p.no == 0) return FP8BW_OK;
   if (p.kc == 0) {
     // An empty contraction: the product is zero (adding it changes nothing).
-    if (p.out_mode == gemm::kOutF32Add) return FP8BW_OK;
-    const size_t esize = gemm::out_is_bf16(p.out_mode) ? 2 : 4;
+    if (p.out_mode == kOutF32Add) return FP8BW_OK;
+    const size_t esize = out_is_bf16(p.out_mode) ? 2 : 4;
     if (cudaMemsetAsync(p.out, 0, static_cast<size_t>(p.mo * p.no) * esize, stream) !=
         cudaSuccess)
       return FP8BW_ERR_CUDA;
-    if (p.out_mode != gemm::kOutBf16Q) return FP8BW_OK;
+    if (p.out_mode != kOutBf16Q) return FP8BW_OK;
     // ... and its row-wise quantisation is that of a zero matrix
     return launch_quantize(kModeRow, false, static_cast<const uint16_t*>(p.out), p.mo, p.no,
                            p.q_out, p.s_out, nullptr, nullptr, nullptr, dev.ordinal, dev.sm_count, stream);
   }
   if (cdiv(p.mo, 256) * cdiv(p.no, 256) > (int64_t(1) << 30)) return FP8BW_ERR_SHAPE;
   if (p.pow2) {
-    if (p.out_mode != gemm::kOutBf16) return FP8BW_ERR_LAUNCH;
+    if (p.vec_b && p.out_mode == kOutF32)
+      return launch_gemm_pow2<true, false, kOutF32>(p, dev, stream);
+    if (p.vec_b && p.out_mode == kOutF32Add)
+      return launch_gemm_pow2<true, false, kOutF32Add>(p, dev, stream);
+    if (p.out_mode != kOutBf16) return FP8BW_ERR_LAUNCH;
     if (p.vec_b) return launch_gemm_pow2<true, false>(p, dev, stream);
     if (p.b_mn) return launch_gemm_pow2<false, true>(p, dev, stream);
     return launch_gemm_pow2<false, false>(p, dev, stream);
   }
-  if (p.vec_b && p.out_mode == gemm::kOutF32)
-    return launch_gemm_pair<GEMM_BN_VEC, true, false, gemm::kOutF32>(p, dev, stream);
-  if (p.vec_b && p.out_mode == gemm::kOutF32Add)
-    return launch_gemm_pair<GEMM_BN_VEC, true, false, gemm::kOutF32Add>(p, dev, stream);
-  if (p.out_mode == gemm::kOutBf16Q && !p.vec_b) {
-    if (p.b_mn) return launch_gemm_pair<256, false, true, gemm::kOutBf16Q>(p, dev, stream);
-    return launch_gemm_pair<256, false, false, gemm::kOutBf16Q>(p, dev, stream);
+  if (p.vec_b && p.out_mode == kOutF32)
+    return launch_gemm_pair<GEMM_BN_VEC, true, false, kOutF32>(p, dev, stream);
+  if (p.vec_b && p.out_mode == kOutF32Add)
+    return launch_gemm_pair<GEMM_BN_VEC, true, false, kOutF32Add>(p, dev, stream);
+  if (p.out_mode == kOutBf16Q && !p.vec_b) {
+    if (p.b_mn) return launch_gemm_pair<256, false, true, kOutBf16Q>(p, dev, stream);
+    return launch_gemm_pair<256, false, false, kOutBf16Q>(p, dev, stream);
   }
-  if (p.out_mode != gemm::kOutBf16) return FP8BW_ERR_LAUNCH;
+  if (p.out_mode != kOutBf16) return FP8BW_ERR_LAUNCH;
   if (p.vec_b) return launch_gemm_pair<GEMM_BN_VEC, true, false>(p, dev, stream);
   if (p.b_mn) return launch_gemm_pair<256, false, true>(p, dev, stream);
   return launch_gemm_pair<GEMM_BN_BLOCK, false, false>(p, dev, stream);
@@ -368,7 +375,7 @@ using namespace fp8bw;
 
 extern "C" {
 
-int fp8bw_version(void) { return 104; }
+int fp8bw_version(void) { return 105; }
 
 const char* fp8bw_status_string(int status) {
   switch (status) {
@@ -538,7 +545,7 @@ int gemm_fprop(bool pow2, const uint8_t* qx, const float* sx, const uint8_t* qw,
   p.pow2 = pow2;
   p.q_out = qy;
   p.s_out = sy;
-  p.out_mode = qy ? gemm::kOutBf16Q : gemm::kOutBf16;
+  p.out_mode = qy ? kOutBf16Q : kOutBf16;
   return run_gemm(p, static_cast<cudaStream_t>(stream));
 }
 
@@ -571,7 +578,7 @@ int gemm_dgrad(bool pow2, const uint8_t* qdy, const float* sdy, const uint8_t* q
   p.pow2 = pow2;
   p.q_out = qdx;
   p.s_out = sdx;
-  p.out_mode = qdx ? gemm::kOutBf16Q : gemm::kOutBf16;
+  p.out_mode = qdx ? kOutBf16Q : kOutBf16;
   return run_gemm(p, static_cast<cudaStream_t>(stream));
 }
 
@@ -633,7 +640,7 @@ int wgrad_common(const uint8_t* qdy_t, const float* sdy_t, const uint8_t* qx_t,
   if (!aligned16(qdy_t) || !aligned16(sdy_t) || !aligned16(qx_t) || !aligned16(sx_t) ||
       !aligned16(dw))
     return FP8BW_ERR_ALIGN;
-  const int64_t esize = gemm::out_is_bf16(out_mode) ? 2 : 4;
+  const int64_t esize = out_is_bf16(out_mode) ? 2 : 4;
   const Range rd = range_of(dw, n * k * esize);
   if (overlap(rd, range_of(qdy_t, n * m)) || overlap(rd, range_of(sdy_t, cdiv(m, 128) * n * 4)) ||
       overlap(rd, range_of(qx_t, k * m)) || overlap(rd, range_of(sx_t, cdiv(m, 128) * k * 4)))
@@ -663,20 +670,27 @@ extern "C" {
 int fp8bw_gemm_wgrad(const uint8_t* qdy_t, const float* sdy_t, const uint8_t* qx_t,
                      const float* sx_t, int64_t m, int64_t n, int64_t k, uint16_t* dw,
                      void* stream) {
-  return wgrad_common(qdy_t, sdy_t, qx_t, sx_t, m, n, k, dw, gemm::kOutBf16, false, stream);
+  return wgrad_common(qdy_t, sdy_t, qx_t, sx_t, m, n, k, dw, kOutBf16, false, stream);
 }
 
 int fp8bw_gemm_wgrad_pow2(const uint8_t* qdy_t, const float* sdy_t, const uint8_t* qx_t,
                           const float* sx_t, int64_t m, int64_t n, int64_t k, uint16_t* dw,
                           void* stream) {
-  return wgrad_common(qdy_t, sdy_t, qx_t, sx_t, m, n, k, dw, gemm::kOutBf16, true, stream);
+  return wgrad_common(qdy_t, sdy_t, qx_t, sx_t, m, n, k, dw, kOutBf16, true, stream);
 }
 
 int fp8bw_gemm_wgrad_f32(const uint8_t* qdy_t, const float* sdy_t, const uint8_t* qx_t,
                          const float* sx_t, int64_t m, int64_t n, int64_t k, float* dw,
                          int accumulate, void* stream) {
   return wgrad_common(qdy_t, sdy_t, qx_t, sx_t, m, n, k, dw,
-                      accumulate ? gemm::kOutF32Add : gemm::kOutF32, false, stream);
+                      accumulate ? kOutF32Add : kOutF32, false, stream);
+}
+
+int fp8bw_gemm_wgrad_f32_pow2(const uint8_t* qdy_t, const float* sdy_t, const uint8_t* qx_t,
+                              const float* sx_t, int64_t m, int64_t n, int64_t k, float* dw,
+                              int accumulate, void* stream) {
+  return wgrad_common(qdy_t, sdy_t, qx_t, sx_t, m, n, k, dw,
+                      accumulate ? kOutF32Add : kOutF32, true, stream);
 }
 
 int fp8bw_selftest_wait_timeout(int64_t limit_ns, void* stream) {

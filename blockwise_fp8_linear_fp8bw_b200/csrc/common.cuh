@@ -52,6 +52,20 @@ int prepare_for_device(DevicePrep& p, int dev, int* value, Fn&& fn) {
 }
 
 // ---------------------------------------------------------------------------
+// Output modes of the GEMM epilogues.
+// ---------------------------------------------------------------------------
+constexpr int kOutBf16 = 0;       // bf16 store
+constexpr int kOutF32 = 1;        // fp32 store
+constexpr int kOutF32Add = 2;     // fp32 add into the existing output (TMA reduce-add)
+constexpr int kOutBf16Q = 3;      // bf16 store + row-wise E4M3 quantisation of that bf16
+                                  // output (block-scale mode only)
+
+// Element type of the output tensor (the TMA map and the staging boxes).
+__host__ __device__ constexpr bool out_is_bf16(int out) {
+  return out == kOutBf16 || out == kOutBf16Q;
+}
+
+// ---------------------------------------------------------------------------
 // Device error record. A kernel whose bounded wait expires ORs a bit in here
 // and returns; fp8bw_check_device_error() reads and clears it.
 // ---------------------------------------------------------------------------

@@ -81,18 +81,6 @@ static_assert(4 * 32 * kProducerRegs + kNumEpiWarps * 32 * kEpilogueRegs ==
                   kThreads * kLaunchRegs,
               "setmaxnreg split must equal the launch register budget");
 
-// Output modes of the epilogue.
-constexpr int kOutBf16 = 0;       // bf16 store
-constexpr int kOutF32 = 1;        // fp32 store
-constexpr int kOutF32Add = 2;     // fp32 add into the existing output (TMA reduce-add)
-constexpr int kOutBf16Q = 3;      // bf16 store + row-wise E4M3 quantisation of that bf16
-                                  // output (block-scale mode only)
-
-// Element type of the output tensor (the TMA map and the staging boxes).
-__host__ __device__ constexpr bool out_is_bf16(int out) {
-  return out == kOutBf16 || out == kOutBf16Q;
-}
-
 struct Args {
   int mo, no, kc;             // output rows, output columns, contraction length
   int tiles_m, tiles_n, chunks;

@@ -33,7 +33,10 @@
 //               is not an exact power of two sets an error bit;
 //   warps 4-11  epilogue: load the 128 x 256 fp32 accumulator from TMEM (each
 //               warp its 32 lanes x 128 columns), release it to the next tile's
-//               MMAs, convert to bf16 and write 32 x 32 boxes with TMA stores.
+//               MMAs, convert to bf16 and write 32 x 32 boxes with TMA stores;
+//               for the weight gradient the fp32 sum can instead leave as fp32
+//               16 x 32 boxes, stored or added element-wise (TMA reduce-add)
+//               into an fp32 tensor already in memory.
 // TMEM: columns 0-255 accumulator, then one 16-column scale-factor slot per
 // ring stage (A: 4 columns, B: 8 columns). Every mbarrier wait is bounded.
 #pragma once
@@ -108,13 +111,15 @@ __device__ __forceinline__ uint32_t ue8m0_word(float s, uint32_t* bad) {
   return e * 0x01010101u;
 }
 
-template <bool VEC_B, bool B_MN>
+template <bool VEC_B, bool B_MN, int OUT = kOutBf16>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     blockwise_gemm_pow2_kernel(const __grid_constant__ CUtensorMap tm_a,
                                const __grid_constant__ CUtensorMap tm_b,
                                const __grid_constant__ CUtensorMap tm_out, const Args g) {
   using L = Layout;
   constexpr int kHalf = BN / 2;                      // columns per epilogue warp
+  static_assert(OUT == kOutBf16 || (VEC_B && (OUT == kOutF32 || OUT == kOutF32Add)),
+                "fp32 outputs are for the weight gradient");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -359,20 +364,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
       const int y0 = tm * (2 * BM) + static_cast<int>(rank) * BM + q * 32;
       const int x0 = tn * BN + h * kHalf;
+      // One 2 KB staging box per warp: 32 rows of 64 bytes (32 bf16 or 16
+      // fp32 columns), 64-byte swizzle (16-byte unit j of row r at j ^ (r/2 % 4)).
+      constexpr int kBoxCols = out_is_bf16(OUT) ? 32 : 16;
 #pragma unroll
-      for (int gi = 0; gi < kHalf / 32; ++gi) {
-        if (x0 + gi * 32 >= g.no || y0 >= g.mo) continue;
+      for (int gi = 0; gi < kHalf / kBoxCols; ++gi) {
+        if (x0 + gi * kBoxCols >= g.no || y0 >= g.mo) continue;
         if (store_pending) {
           if (lane == 0) bulk_wait_group_read<0>();
           __syncwarp();
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const uint32_t* v = r + gi * 32 + j * 8;
-          const uint32_t w0 = pack_bf16x2(__uint_as_float(v[0]), __uint_as_float(v[1]));
-          const uint32_t w1 = pack_bf16x2(__uint_as_float(v[2]), __uint_as_float(v[3]));
-          const uint32_t w2 = pack_bf16x2(__uint_as_float(v[4]), __uint_as_float(v[5]));
-          const uint32_t w3 = pack_bf16x2(__uint_as_float(v[6]), __uint_as_float(v[7]));
+          uint32_t w0, w1, w2, w3;
+          if constexpr (out_is_bf16(OUT)) {
+            const uint32_t* v = r + gi * 32 + j * 8;
+            w0 = pack_bf16x2(__uint_as_float(v[0]), __uint_as_float(v[1]));
+            w1 = pack_bf16x2(__uint_as_float(v[2]), __uint_as_float(v[3]));
+            w2 = pack_bf16x2(__uint_as_float(v[4]), __uint_as_float(v[5]));
+            w3 = pack_bf16x2(__uint_as_float(v[6]), __uint_as_float(v[7]));
+          } else {
+            const uint32_t* v = r + gi * 16 + j * 4;
+            w0 = v[0];
+            w1 = v[1];
+            w2 = v[2];
+            w3 = v[3];
+          }
           const uint32_t dst = stage_out + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4);
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(w0), "r"(w1),
                        "r"(w2), "r"(w3)
@@ -381,7 +398,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&tm_out, stage_out, x0 + gi * 32, y0);
+          if constexpr (OUT == kOutF32Add)
+            tma_reduce_add_2d(&tm_out, stage_out, x0 + gi * kBoxCols, y0);
+          else
+            tma_store_2d(&tm_out, stage_out, x0 + gi * kBoxCols, y0);
           bulk_commit_group();
         }
         store_pending = true;

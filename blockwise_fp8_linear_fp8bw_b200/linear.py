@@ -13,9 +13,8 @@ hidden flow, fp32 gradients):
             dX = dgrad(dY, W)                                      bf16
             dW = wgrad(dY, X): added in fp32 into weight.main_grad when the
                  weight carries one (gradient accumulation over
-                 micro-batches), else returned in the weight's dtype.
-                 The power-of-two-scale wgrad writes bf16 only, so on that
-                 path the bf16 dW is widened and then added to main_grad.
+                 micro-batches; the add is done by the GEMM's epilogue, for
+                 either scale form), else returned in the weight's dtype.
 
 Every step runs in the CUDA library; this module only reshapes tensors and
 keeps the codes the backward pass needs. Inputs must be bf16 CUDA tensors
@@ -66,11 +65,9 @@ class BlockwiseFp8LinearFunction(torch.autograd.Function):
                                 pow2=ctx.pow2).reshape(ctx.x_shape)
         if ctx.needs_input_grad[1]:
             main = getattr(weight, "main_grad", None)
-            if main is not None and not ctx.pow2:
-                ops.gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, main_grad=main)
-            elif main is not None:
-                main += ops.gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t,
-                                       pow2=True).float()
+            if main is not None:
+                ops.gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, main_grad=main,
+                                   pow2=ctx.pow2)
             else:
                 dw = ops.gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t, pow2=ctx.pow2)
                 if dw.dtype != weight.dtype:

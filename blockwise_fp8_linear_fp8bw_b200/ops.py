@@ -181,7 +181,7 @@ def fp8bw_gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t, dw, stream=None, pow2=False):
 
 
 def fp8bw_gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, dw, accumulate=False,
-                         stream=None):
+                         stream=None, pow2=False):
     n, m = qdy_t.shape
     k = qx_t.shape[0]
     _expect(qdy_t, torch.uint8, (n, m), "qdy_t")
@@ -189,8 +189,8 @@ def fp8bw_gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, dw, accumulate=False,
     _expect(sdy_t, torch.float32, (_cdiv(m, 128), n), "sdy_t")
     _expect(sx_t, torch.float32, (_cdiv(m, 128), k), "sx_t")
     _expect(dw, torch.float32, (n, k), "dw")
-    _call("fp8bw_gemm_wgrad_f32", (qdy_t, sdy_t, qx_t, sx_t, dw), stream,
-          _ptr(qdy_t), _ptr(sdy_t), _ptr(qx_t), _ptr(sx_t), m, n, k,
+    _call(_fn("fp8bw_gemm_wgrad_f32", pow2), (qdy_t, sdy_t, qx_t, sx_t, dw),
+          stream, _ptr(qdy_t), _ptr(sdy_t), _ptr(qx_t), _ptr(sx_t), m, n, k,
           _ptr(dw), 1 if accumulate else 0)
 
 
@@ -320,15 +320,17 @@ def gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t, stream=None, pow2=False):
     return dw
 
 
-def gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, main_grad=None, stream=None):
+def gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, main_grad=None, stream=None,
+                   pow2=False):
     """fp32 dW; with `main_grad` given, dW is added into it in place and it is
     returned."""
     if main_grad is not None:
-        fp8bw_gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, main_grad, True, stream)
+        fp8bw_gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, main_grad, True, stream,
+                             pow2=pow2)
         return main_grad
     dw = torch.empty((qdy_t.shape[0], qx_t.shape[0]), dtype=torch.float32,
                      device=qdy_t.device)
-    fp8bw_gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, dw, False, stream)
+    fp8bw_gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, dw, False, stream, pow2=pow2)
     return dw
 
 

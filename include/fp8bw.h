@@ -227,6 +227,19 @@ int fp8bw_gemm_wgrad_pow2(const uint8_t* qdy_t, const float* sdy_t,
                           const uint8_t* qx_t, const float* sx_t, int64_t m,
                           int64_t n, int64_t k, uint16_t* dw, void* stream);
 
+/* Power-of-two wgrad with an fp32 weight gradient (the power-of-two form of
+ * fp8bw_gemm_wgrad_f32): the fp32 sum that fp8bw_gemm_wgrad_pow2 rounds to
+ * bf16, stored (accumulate == 0) or added
+ * element-wise into dw (accumulate != 0: dW := fp32(dW + P), one add per
+ * element by the TMA unit), as fp8bw_gemm_wgrad_f32 does for the other scale
+ * form. dw: fp32 [n, k], caller-owned, 16-byte aligned, not overlapping any
+ * input. Source: paperlayer.ai summary, Appendix C, "FP8 implementation
+ * pipeline" (gradients kept in FP32). */
+int fp8bw_gemm_wgrad_f32_pow2(const uint8_t* qdy_t, const float* sdy_t,
+                              const uint8_t* qx_t, const float* sx_t,
+                              int64_t m, int64_t n, int64_t k, float* dw,
+                              int accumulate, void* stream);
+
 /* Synchronises `stream`, then returns FP8BW_ERR_DEVICE_TIMEOUT if any kernel
  * of this library on the current device recorded an expired wait since the
  * last call, FP8BW_ERR_SCALE if a *_pow2 GEMM recorded a scale that is not a
