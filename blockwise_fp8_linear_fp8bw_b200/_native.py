@@ -27,6 +27,10 @@ SIGNATURES = {
                                 _P], _INT),
     "fp8bw_gemm_dgrad_quant": ([_P, _P, _P, _INT, _P, _I64, _I64, _I64, _P, _P,
                                 _P, _P], _INT),
+    "fp8bw_gemm_fprop_quant_rowcol": ([_P, _P, _P, _P, _I64, _I64, _I64, _P, _P,
+                                       _P, _P, _P, _P], _INT),
+    "fp8bw_gemm_dgrad_quant_rowcol": ([_P, _P, _P, _INT, _P, _I64, _I64, _I64, _P,
+                                       _P, _P, _P, _P, _P], _INT),
     "fp8bw_quantize_rowwise_pow2": ([_P, _I64, _I64, _P, _P, _P], _INT),
     "fp8bw_quantize_colwise_pow2": ([_P, _I64, _I64, _P, _P, _P, _P, _P], _INT),
     "fp8bw_quantize_weight_block_pow2": ([_P, _I64, _I64, _P, _P, _P, _P], _INT),

@@ -196,8 +196,10 @@ struct GemmProblem {
   void* out;         // [mo][no]: bf16 (kOutBf16) or fp32
   int out_mode;      // kOutBf16 / kOutF32 / kOutF32Add
   bool pow2;         // power-of-two scales on the hardware block-scaled MMA
-  uint8_t* q_out;    // kOutBf16Q: row-wise codes of the bf16 output [mo][no]
-  float* s_out;      // kOutBf16Q: their scales [ceil(no/128)][mo]
+  uint8_t* q_out;    // kOutBf16Q(Q): row-wise codes of the bf16 output [mo][no]
+  float* s_out;      // kOutBf16Q(Q): their scales [ceil(no/128)][mo]
+  uint8_t* qt_out;   // kOutBf16QQ: column-wise codes, transposed [no][mo]
+  float* st_out;     // kOutBf16QQ: their scales [ceil(mo/128)][no]
 };
 
 // CTA-pair kernel: 256 x 256 output tiles on clusters of two CTAs.
@@ -255,6 +257,8 @@ int launch_gemm_pair(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t s
   g.out = p.out;
   g.q_out = p.q_out;
   g.s_out = p.s_out;
+  g.qt_out = p.qt_out;
+  g.st_out = p.st_out;
   const int64_t tiles = static_cast<int64_t>(g.tiles_m) * g.tiles_n;
   const int clusters = static_cast<int>(std::min<int64_t>(tiles, max_clusters));
   kernel<<<2 * clusters, gemm::kThreads, L::kAlloc, stream>>>(tm_a, tm_b, tm_out, g);
@@ -338,8 +342,12 @@ int run_gemm(const GemmProblem& p, cudaStream_t stream) {
     if (cudaMemsetAsync(p.out, 0, static_cast<size_t>(p.mo * p.no) * esize, stream) !=
         cudaSuccess)
       return FP8BW_ERR_CUDA;
-    if (p.out_mode != kOutBf16Q) return FP8BW_OK;
-    // ... and its row-wise quantisation is that of a zero matrix
+    if (!out_quant_rows(p.out_mode)) return FP8BW_OK;
+    // ... and its quantisation is that of a zero matrix
+    if (p.out_mode == kOutBf16QQ)
+      return launch_quantize(kModeRowCol, false, static_cast<const uint16_t*>(p.out), p.mo, p.no,
+                             p.q_out, p.s_out, p.qt_out, p.st_out, nullptr, dev.ordinal,
+                             dev.sm_count, stream);
     return launch_quantize(kModeRow, false, static_cast<const uint16_t*>(p.out), p.mo, p.no,
                            p.q_out, p.s_out, nullptr, nullptr, nullptr, dev.ordinal, dev.sm_count, stream);
   }
@@ -362,6 +370,10 @@ int run_gemm(const GemmProblem& p, cudaStream_t stream) {
     if (p.b_mn) return launch_gemm_pair<256, false, true, kOutBf16Q>(p, dev, stream);
     return launch_gemm_pair<256, false, false, kOutBf16Q>(p, dev, stream);
   }
+  if (p.out_mode == kOutBf16QQ && !p.vec_b) {
+    if (p.b_mn) return launch_gemm_pair<256, false, true, kOutBf16QQ>(p, dev, stream);
+    return launch_gemm_pair<256, false, false, kOutBf16QQ>(p, dev, stream);
+  }
   if (p.out_mode != kOutBf16) return FP8BW_ERR_LAUNCH;
   if (p.vec_b) return launch_gemm_pair<GEMM_BN_VEC, true, false>(p, dev, stream);
   if (p.b_mn) return launch_gemm_pair<256, false, true>(p, dev, stream);
@@ -375,7 +387,7 @@ using namespace fp8bw;
 
 extern "C" {
 
-int fp8bw_version(void) { return 105; }
+int fp8bw_version(void) { return 106; }
 
 const char* fp8bw_status_string(int status) {
   switch (status) {
@@ -505,20 +517,26 @@ namespace {
 // its row-wise quantisation (q [rows, cols], s [ceil(cols/128)][rows]):
 // alignment, and no overlap with the inputs or with each other.
 int quant_outputs_status(const void* out, int64_t rows, int64_t cols, const uint8_t* q,
-                         const float* s, const Range* ins, int nins) {
-  if (!aligned16(q) || !aligned16(s)) return FP8BW_ERR_ALIGN;
-  const Range ro = range_of(out, rows * cols * 2);
-  const Range rq = range_of(q, q ? rows * cols : 0);
-  const Range rs = range_of(s, s ? cdiv(cols, 128) * rows * 4 : 0);
-  for (int i = 0; i < nins; ++i)
-    if (overlap(ro, ins[i]) || overlap(rq, ins[i]) || overlap(rs, ins[i])) return FP8BW_ERR_ALIAS;
-  if (overlap(ro, rq) || overlap(ro, rs) || overlap(rq, rs)) return FP8BW_ERR_ALIAS;
+                         const float* s, const Range* ins, int nins,
+                         const uint8_t* q_t = nullptr, const float* s_t = nullptr) {
+  if (!aligned16(q) || !aligned16(s) || !aligned16(q_t) || !aligned16(s_t))
+    return FP8BW_ERR_ALIGN;
+  const Range outs[5] = {range_of(out, rows * cols * 2), range_of(q, q ? rows * cols : 0),
+                         range_of(s, s ? cdiv(cols, 128) * rows * 4 : 0),
+                         range_of(q_t, q_t ? rows * cols : 0),
+                         range_of(s_t, s_t ? cdiv(rows, 128) * cols * 4 : 0)};
+  for (int o = 0; o < 5; ++o) {
+    for (int i = 0; i < nins; ++i)
+      if (overlap(outs[o], ins[i])) return FP8BW_ERR_ALIAS;
+    for (int o2 = o + 1; o2 < 5; ++o2)
+      if (overlap(outs[o], outs[o2])) return FP8BW_ERR_ALIAS;
+  }
   return FP8BW_OK;
 }
 
 int gemm_fprop(bool pow2, const uint8_t* qx, const float* sx, const uint8_t* qw, const float* sw,
                int64_t m, int64_t n, int64_t k, uint16_t* y, uint8_t* qy, float* sy,
-               void* stream) {
+               void* stream, uint8_t* qy_t = nullptr, float* sy_t = nullptr) {
   if (!dim_ok(m) || !dim_ok(n) || !dim_ok(k)) return FP8BW_ERR_SHAPE;
   if (missing(qx, m * k) || missing(sx, cdiv(k, 128) * m) || missing(qw, n * k) ||
       missing(sw, cdiv(n, 128) * cdiv(k, 128)) || missing(y, m * n))
@@ -527,7 +545,7 @@ int gemm_fprop(bool pow2, const uint8_t* qx, const float* sx, const uint8_t* qw,
     return FP8BW_ERR_ALIGN;
   const Range ins[4] = {range_of(qx, m * k), range_of(sx, cdiv(k, 128) * m * 4),
                         range_of(qw, n * k), range_of(sw, cdiv(n, 128) * cdiv(k, 128) * 4)};
-  const int ost = quant_outputs_status(y, m, n, qy, sy, ins, 4);
+  const int ost = quant_outputs_status(y, m, n, qy, sy, ins, 4, qy_t, sy_t);
   if (ost != FP8BW_OK) return ost;
   GemmProblem p{};
   p.a = qx;
@@ -545,13 +563,16 @@ int gemm_fprop(bool pow2, const uint8_t* qx, const float* sx, const uint8_t* qw,
   p.pow2 = pow2;
   p.q_out = qy;
   p.s_out = sy;
-  p.out_mode = qy ? kOutBf16Q : kOutBf16;
+  p.qt_out = qy_t;
+  p.st_out = sy_t;
+  p.out_mode = qy_t ? kOutBf16QQ : (qy ? kOutBf16Q : kOutBf16);
   return run_gemm(p, static_cast<cudaStream_t>(stream));
 }
 
 int gemm_dgrad(bool pow2, const uint8_t* qdy, const float* sdy, const uint8_t* qw,
                int qw_is_transposed, const float* sw, int64_t m, int64_t n, int64_t k,
-               uint16_t* dx, uint8_t* qdx, float* sdx, void* stream) {
+               uint16_t* dx, uint8_t* qdx, float* sdx, void* stream, uint8_t* qdx_t = nullptr,
+               float* sdx_t = nullptr) {
   if (!dim_ok(m) || !dim_ok(n) || !dim_ok(k)) return FP8BW_ERR_SHAPE;
   if (missing(qdy, m * n) || missing(sdy, cdiv(n, 128) * m) || missing(qw, n * k) ||
       missing(sw, cdiv(n, 128) * cdiv(k, 128)) || missing(dx, m * k))
@@ -560,7 +581,7 @@ int gemm_dgrad(bool pow2, const uint8_t* qdy, const float* sdy, const uint8_t* q
     return FP8BW_ERR_ALIGN;
   const Range ins[4] = {range_of(qdy, m * n), range_of(sdy, cdiv(n, 128) * m * 4),
                         range_of(qw, n * k), range_of(sw, cdiv(n, 128) * cdiv(k, 128) * 4)};
-  const int ost = quant_outputs_status(dx, m, k, qdx, sdx, ins, 4);
+  const int ost = quant_outputs_status(dx, m, k, qdx, sdx, ins, 4, qdx_t, sdx_t);
   if (ost != FP8BW_OK) return ost;
   GemmProblem p{};
   p.a = qdy;
@@ -578,7 +599,9 @@ int gemm_dgrad(bool pow2, const uint8_t* qdy, const float* sdy, const uint8_t* q
   p.pow2 = pow2;
   p.q_out = qdx;
   p.s_out = sdx;
-  p.out_mode = qdx ? kOutBf16Q : kOutBf16;
+  p.qt_out = qdx_t;
+  p.st_out = sdx_t;
+  p.out_mode = qdx_t ? kOutBf16QQ : (qdx ? kOutBf16Q : kOutBf16);
   return run_gemm(p, static_cast<cudaStream_t>(stream));
 }
 
@@ -612,6 +635,31 @@ int fp8bw_gemm_dgrad_quant(const uint8_t* qdy, const float* sdy, const uint8_t* 
   if (missing(qdx, m * k) || missing(sdx, cdiv(k, 128) * m)) return FP8BW_ERR_NULL;
   if (m * k > 0 && (qdx == nullptr || sdx == nullptr)) return FP8BW_ERR_NULL;
   return gemm_dgrad(false, qdy, sdy, qw, qw_is_transposed, sw, m, n, k, dx, qdx, sdx, stream);
+}
+
+int fp8bw_gemm_fprop_quant_rowcol(const uint8_t* qx, const float* sx, const uint8_t* qw,
+                                  const float* sw, int64_t m, int64_t n, int64_t k, uint16_t* y,
+                                  uint8_t* qy, float* sy, uint8_t* qy_t, float* sy_t,
+                                  void* stream) {
+  if (missing(qy, m * n) || missing(sy, cdiv(n, 128) * m) || missing(qy_t, m * n) ||
+      missing(sy_t, cdiv(m, 128) * n))
+    return FP8BW_ERR_NULL;
+  if (m * n > 0 && (qy == nullptr || sy == nullptr || qy_t == nullptr || sy_t == nullptr))
+    return FP8BW_ERR_NULL;
+  return gemm_fprop(false, qx, sx, qw, sw, m, n, k, y, qy, sy, stream, qy_t, sy_t);
+}
+
+int fp8bw_gemm_dgrad_quant_rowcol(const uint8_t* qdy, const float* sdy, const uint8_t* qw,
+                                  int qw_is_transposed, const float* sw, int64_t m, int64_t n,
+                                  int64_t k, uint16_t* dx, uint8_t* qdx, float* sdx,
+                                  uint8_t* qdx_t, float* sdx_t, void* stream) {
+  if (missing(qdx, m * k) || missing(sdx, cdiv(k, 128) * m) || missing(qdx_t, m * k) ||
+      missing(sdx_t, cdiv(m, 128) * k))
+    return FP8BW_ERR_NULL;
+  if (m * k > 0 && (qdx == nullptr || sdx == nullptr || qdx_t == nullptr || sdx_t == nullptr))
+    return FP8BW_ERR_NULL;
+  return gemm_dgrad(false, qdy, sdy, qw, qw_is_transposed, sw, m, n, k, dx, qdx, sdx, stream,
+                    qdx_t, sdx_t);
 }
 
 int fp8bw_gemm_fprop_pow2(const uint8_t* qx, const float* sx, const uint8_t* qw, const float* sw,

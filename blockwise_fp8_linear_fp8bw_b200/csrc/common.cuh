@@ -59,10 +59,17 @@ constexpr int kOutF32 = 1;        // fp32 store
 constexpr int kOutF32Add = 2;     // fp32 add into the existing output (TMA reduce-add)
 constexpr int kOutBf16Q = 3;      // bf16 store + row-wise E4M3 quantisation of that bf16
                                   // output (block-scale mode only)
+constexpr int kOutBf16QQ = 4;     // bf16 store + row-wise and column-wise (transposed)
+                                  // E4M3 quantisation of it (block-scale mode only)
 
 // Element type of the output tensor (the TMA map and the staging boxes).
 __host__ __device__ constexpr bool out_is_bf16(int out) {
-  return out == kOutBf16 || out == kOutBf16Q;
+  return out == kOutBf16 || out == kOutBf16Q || out == kOutBf16QQ;
+}
+
+// Output modes that also quantise the bf16 output row-wise.
+__host__ __device__ constexpr bool out_quant_rows(int out) {
+  return out == kOutBf16Q || out == kOutBf16QQ;
 }
 
 // ---------------------------------------------------------------------------

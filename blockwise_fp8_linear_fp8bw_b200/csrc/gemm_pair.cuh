@@ -89,8 +89,10 @@ struct Args {
   int64_t sbj, sbc;
   int nblk;                   // number of 128-wide output column blocks
   void* out;                  // [mo][no], bf16 or fp32 (written through tm_out)
-  uint8_t* q_out;             // kOutBf16Q: codes [mo][no]
-  float* s_out;               // kOutBf16Q: scales [ceil(no/128)][mo]
+  uint8_t* q_out;             // kOutBf16Q(Q): codes [mo][no]
+  float* s_out;               // kOutBf16Q(Q): scales [ceil(no/128)][mo]
+  uint8_t* qt_out;            // kOutBf16QQ: transposed column-wise codes [no][mo]
+  float* st_out;              // kOutBf16QQ: their scales [ceil(mo/128)][no]
 };
 
 __device__ __forceinline__ void setmaxnreg_dec() {
@@ -120,11 +122,15 @@ struct PairLayout {
   static constexpr int kScaleSlot = kSaBytes + kSbBytes;
   static constexpr int kScaleOff = kRingBytes;
   static constexpr int kBarOff = kScaleOff + kScaleStages * kScaleSlot;
-  static constexpr int kNumBars = 2 * kStages + 2 * kScaleStages + 2 * kTmemBufs + 1;
+  // + 2 x 2 column-max barriers (column half, double buffer) for kOutBf16QQ
+  static constexpr int kNumBars = 2 * kStages + 2 * kScaleStages + 2 * kTmemBufs + 1 + 4;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kOutWarpBytes = 32 * 32 * 2;
   static constexpr int kOutOff = ((kMiscOff + 16 + 1023) / 1024) * 1024;
-  static constexpr int kBytes = kOutOff + kNumEpiWarps * kOutWarpBytes;
+  // kOutBf16QQ: per column half and buffer, 4 warps x 32 column maxima
+  static constexpr int kColMaxOff = kOutOff + kNumEpiWarps * kOutWarpBytes;
+  static constexpr int kColMaxBytes = 2 * 2 * 4 * 32 * 4;
+  static constexpr int kBytes = kColMaxOff + kColMaxBytes;
   static constexpr int kAlloc = kBytes + 1024;
   static constexpr uint32_t kTmemCols = 512;     // kTmemBufs x BN columns
   static_assert(kAlloc <= 227 * 1024, "shared memory budget");
@@ -141,7 +147,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   constexpr int kPairStages = L::kStages;
   constexpr int kBufs = L::kTmemBufs;
   static_assert(!B_MN || BN == 256, "MN-major B uses full 128-element swizzle atoms");
-  static_assert(OUT != kOutBf16Q || (!VEC_B && BN == 256),
+  static_assert(!out_quant_rows(OUT) || (!VEC_B && BN == 256),
                 "the fused quantisation needs one 128-column group per thread");
   constexpr int kHalf = BN / 2;                      // columns per epilogue thread
   constexpr uint32_t kIdesc = idesc_e4m3(2 * BM, BN, B_MN);
@@ -160,6 +166,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     return bar0 + 8u * (2 * kPairStages + 2 * kScaleStages + kBufs + b);
   };
   const uint32_t drain_bar = bar0 + 8u * (2 * kPairStages + 2 * kScaleStages + 2 * kBufs);
+  // kOutBf16QQ: the four warps of column half hh meet here, box by box
+  auto colmax_bar = [&](int hh, int b) { return drain_bar + 8u * (1 + 2 * hh + b); };
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L::kMiscOff);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
@@ -182,6 +190,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(tempty_bar(b), 2 * kNumEpiWarps);  // used on the leader only
     }
     mbar_init(drain_bar, 1);
+    for (int b = 0; b < 4; ++b) mbar_init(colmax_bar(b >> 1, b & 1), 4);
     *abort_flag = 0u;
     fence_mbar_init();
   }
@@ -367,6 +376,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t stage_out = sbase + L::kOutOff + ew * L::kOutWarpBytes;
     const uint32_t tempty_leader0 = mapa_shared(tempty_bar(0), 0);
     uint32_t tc = 0, sit = 0;
+    uint32_t box_seq = 0;         // kOutBf16QQ: boxes this warp has quantised
     bool ok = true, store_pending = false;
     for (int tile = cluster_id; ok && tile < num_tiles; tile += num_clusters) {
       const int tm = tile / g.tiles_n, tn = tile % g.tiles_n;
@@ -468,7 +478,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // group (x0 is a multiple of 128) of the bf16 output; quantise the bf16
       // values as the row-wise quantiser would.
       float qscale = 1.0f;
-      if constexpr (OUT == kOutBf16Q) {
+      if constexpr (out_quant_rows(OUT)) {
         uint32_t mx = 0u;
 #pragma unroll
         for (int j = 0; j < kHalf / 2; ++j)
@@ -483,7 +493,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       constexpr int kBoxCols = out_is_bf16(OUT) ? 32 : 16;
 #pragma unroll
       for (int gi = 0; gi < kHalf / kBoxCols; ++gi) {
-        if (x0 + gi * kBoxCols >= g.no || y0 >= g.mo) continue;
+        // kOutBf16QQ: the four warps of this column half exchange column
+        // maxima for every box that has columns in range, so a warp whose
+        // rows are all past the end still takes part (it stores nothing).
+        if (x0 + gi * kBoxCols >= g.no) continue;
+        if (OUT != kOutBf16QQ && y0 >= g.mo) continue;
         if (store_pending) {
           if (lane == 0) bulk_wait_group_read<0>();
           __syncwarp();
@@ -517,7 +531,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
           }
         } else {
-          uint32_t codes[8];   // kOutBf16Q: this row's 32 codes of the box
+          uint32_t codes[8];   // row-wise: this row's 32 codes of the box
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             uint32_t w0, w1, w2, w3;
@@ -527,7 +541,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               w1 = pack_bf16x2(v[2], v[3]);
               w2 = pack_bf16x2(v[4], v[5]);
               w3 = pack_bf16x2(v[6], v[7]);
-              if constexpr (OUT == kOutBf16Q) {
+              if constexpr (out_quant_rows(OUT)) {
                 float t[8];
                 scale_pair(w0, qscale, t[0], t[1]);
                 scale_pair(w1, qscale, t[2], t[3]);
@@ -548,7 +562,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                          "r"(w1), "r"(w2), "r"(w3)
                          : "memory");
           }
-          if constexpr (OUT == kOutBf16Q) {
+          if constexpr (out_quant_rows(OUT)) {
             const int grow = y0 + lane;
             if (grow < g.mo) {
               uint8_t* dst = g.q_out + static_cast<int64_t>(grow) * g.no + x0 + gi * 32;
@@ -557,6 +571,67 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 *reinterpret_cast<uint4*>(dst + 16) =
                     make_uint4(codes[4], codes[5], codes[6], codes[7]);
             }
+          }
+          if constexpr (OUT == kOutBf16QQ) {
+            // Column-wise 128x1 groups of the bf16 output: this CTA's 128 rows
+            // are exactly one token group (its first row is a multiple of
+            // 128). Lane l takes column l of this warp's staged box (32
+            // tokens), the four warps of the column half combine their maxima
+            // through shared memory, and each thread encodes its 32 tokens of
+            // the column into the transposed codes. Rows past the end are
+            // zero (the operand loads read zeros there), as a short last group
+            // reads as zero-padded.
+            __syncwarp();
+            uint32_t cv[16];     // column `lane`, rows 2i and 2i+1 as a bf16 pair
+            uint32_t m2 = 0u;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              uint32_t v2[2];
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int rr = 2 * i + e;
+                const uint32_t addr = stage_out + rr * 64 +
+                                      (((lane >> 3) ^ ((rr >> 1) & 3)) << 4) + (lane & 7) * 2;
+                uint16_t hv;
+                asm volatile("ld.shared.u16 %0, [%1];" : "=h"(hv) : "r"(addr) : "memory");
+                v2[e] = hv;
+              }
+              cv[i] = v2[0] | (v2[1] << 16);
+              m2 = max_bf16x2(m2, abs_bf16x2(cv[i]));
+            }
+            const int cb = static_cast<int>(box_seq & 1u);
+            const uint32_t cph = (box_seq >> 1) & 1u;
+            ++box_seq;
+            float* cmax = reinterpret_cast<float*>(smem + L::kColMaxOff) + (h * 2 + cb) * 128;
+            cmax[q * 32 + lane] = max_halves(m2);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(colmax_bar(h, cb));
+            if (!mbar_wait(colmax_bar(h, cb), cph, abort_flag, kErrTimeoutEpi)) {
+              ok = false;
+              break;
+            }
+            const float amax = fmaxf(fmaxf(cmax[lane], cmax[32 + lane]),
+                                     fmaxf(cmax[64 + lane], cmax[96 + lane]));
+            float cqs, csc;
+            group_scale(amax, cqs, csc);
+            const int col = x0 + gi * 32 + lane;
+            const int tg = tm * 2 + static_cast<int>(rank);     // token group
+            if (col < g.no) {
+              if (q == 0 && tg * 128 < g.mo) g.st_out[static_cast<int64_t>(tg) * g.no + col] = csc;
+              uint32_t cc[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                float t[4];
+                scale_pair(cv[2 * i], cqs, t[0], t[1]);
+                scale_pair(cv[2 * i + 1], cqs, t[2], t[3]);
+                cc[i] = e4m3x2(t[0], t[1]) | (e4m3x2(t[2], t[3]) << 16);
+              }
+              uint8_t* dst = g.qt_out + static_cast<int64_t>(col) * g.mo + y0;
+              if (y0 < g.mo) *reinterpret_cast<uint4*>(dst) = make_uint4(cc[0], cc[1], cc[2], cc[3]);
+              if (y0 + 16 < g.mo)
+                *reinterpret_cast<uint4*>(dst + 16) = make_uint4(cc[4], cc[5], cc[6], cc[7]);
+            }
+            if (y0 >= g.mo) continue;       // nothing of this warp's box to store
           }
         }
         fence_proxy_async_smem();
@@ -570,6 +645,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         store_pending = true;
       }
+      if (!ok) break;
     }
     if (lane == 0) bulk_wait_group_all();
   }

@@ -225,6 +225,44 @@ def fp8bw_gemm_dgrad_quant(qdy, sdy, qw, qw_is_transposed, sw, dx, qdx, sdx,
           _ptr(sw), m, n, k, _ptr(dx), _ptr(qdx), _ptr(sdx))
 
 
+def fp8bw_gemm_fprop_quant_rowcol(qx, sx, qw, sw, y, qy, sy, qy_t, sy_t,
+                                  stream=None):
+    m, k = qx.shape
+    n = qw.shape[0]
+    _expect(qx, torch.uint8, (m, k), "qx")
+    _expect(qw, torch.uint8, (n, k), "qw")
+    _expect(sx, torch.float32, (_cdiv(k, 128), m), "sx")
+    _expect(sw, torch.float32, (_cdiv(n, 128), _cdiv(k, 128)), "sw")
+    _expect(y, torch.bfloat16, (m, n), "y")
+    _expect(qy, torch.uint8, (m, n), "qy")
+    _expect(sy, torch.float32, (_cdiv(n, 128), m), "sy")
+    _expect(qy_t, torch.uint8, (n, m), "qy_t")
+    _expect(sy_t, torch.float32, (_cdiv(m, 128), n), "sy_t")
+    _call("fp8bw_gemm_fprop_quant_rowcol", (qx, sx, qw, sw, y, qy, sy, qy_t, sy_t),
+          stream, _ptr(qx), _ptr(sx), _ptr(qw), _ptr(sw), m, n, k, _ptr(y),
+          _ptr(qy), _ptr(sy), _ptr(qy_t), _ptr(sy_t))
+
+
+def fp8bw_gemm_dgrad_quant_rowcol(qdy, sdy, qw, qw_is_transposed, sw, dx, qdx,
+                                  sdx, qdx_t, sdx_t, stream=None):
+    m, n = qdy.shape
+    k = qw.shape[0] if qw_is_transposed else qw.shape[1]
+    _expect(qdy, torch.uint8, (m, n), "qdy")
+    _expect(qw, torch.uint8, (k, n) if qw_is_transposed else (n, k), "qw")
+    _expect(sdy, torch.float32, (_cdiv(n, 128), m), "sdy")
+    _expect(sw, torch.float32, (_cdiv(n, 128), _cdiv(k, 128)), "sw")
+    _expect(dx, torch.bfloat16, (m, k), "dx")
+    _expect(qdx, torch.uint8, (m, k), "qdx")
+    _expect(sdx, torch.float32, (_cdiv(k, 128), m), "sdx")
+    _expect(qdx_t, torch.uint8, (k, m), "qdx_t")
+    _expect(sdx_t, torch.float32, (_cdiv(m, 128), k), "sdx_t")
+    _call("fp8bw_gemm_dgrad_quant_rowcol",
+          (qdy, sdy, qw, sw, dx, qdx, sdx, qdx_t, sdx_t), stream,
+          _ptr(qdy), _ptr(sdy), _ptr(qw), 1 if qw_is_transposed else 0,
+          _ptr(sw), m, n, k, _ptr(dx), _ptr(qdx), _ptr(sdx), _ptr(qdx_t),
+          _ptr(sdx_t))
+
+
 def _device_call(name, stream, device, *args):
     """Call a device-wide entry point (no tensor arguments) for one device:
     `device` if given, else the device of a torch `stream`, else the current
@@ -356,3 +394,34 @@ def gemm_dgrad_quant(qdy, sdy, qw, sw, qw_is_transposed=True, stream=None):
     fp8bw_gemm_dgrad_quant(qdy, sdy, qw, qw_is_transposed, sw, dx, qdx, sdx,
                            stream)
     return dx, qdx, sdx
+
+
+def gemm_fprop_quant_rowcol(qx, sx, qw, sw, stream=None):
+    """-> (y, qy, sy, qy_t, sy_t): the bf16 product with its row-wise and its
+    transposed column-wise quantisation."""
+    m, n = qx.shape[0], qw.shape[0]
+    dev = qx.device
+    y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+    qy = torch.empty((m, n), dtype=torch.uint8, device=dev)
+    sy = torch.empty((_cdiv(n, 128), m), dtype=torch.float32, device=dev)
+    qy_t = torch.empty((n, m), dtype=torch.uint8, device=dev)
+    sy_t = torch.empty((_cdiv(m, 128), n), dtype=torch.float32, device=dev)
+    fp8bw_gemm_fprop_quant_rowcol(qx, sx, qw, sw, y, qy, sy, qy_t, sy_t, stream)
+    return y, qy, sy, qy_t, sy_t
+
+
+def gemm_dgrad_quant_rowcol(qdy, sdy, qw, sw, qw_is_transposed=True,
+                            stream=None):
+    """-> (dx, qdx, sdx, qdx_t, sdx_t): the bf16 product with its row-wise
+    and its transposed column-wise quantisation."""
+    m = qdy.shape[0]
+    k = qw.shape[0] if qw_is_transposed else qw.shape[1]
+    dev = qdy.device
+    dx = torch.empty((m, k), dtype=torch.bfloat16, device=dev)
+    qdx = torch.empty((m, k), dtype=torch.uint8, device=dev)
+    sdx = torch.empty((_cdiv(k, 128), m), dtype=torch.float32, device=dev)
+    qdx_t = torch.empty((k, m), dtype=torch.uint8, device=dev)
+    sdx_t = torch.empty((_cdiv(m, 128), k), dtype=torch.float32, device=dev)
+    fp8bw_gemm_dgrad_quant_rowcol(qdy, sdy, qw, qw_is_transposed, sw, dx, qdx,
+                                  sdx, qdx_t, sdx_t, stream)
+    return dx, qdx, sdx, qdx_t, sdx_t

@@ -189,6 +189,36 @@ int fp8bw_gemm_dgrad_quant(const uint8_t* qdy, const float* sdy,
                            uint16_t* dx, uint8_t* qdx, float* sdx,
                            void* stream);
 
+/* fprop / dgrad that quantise their own bf16 output both ways, as
+ * fp8bw_quantize_colwise with q_row/s_row would: the row-wise codes and
+ * scales of the calls above, plus the column-wise 128x1 codes written
+ * transposed and their scales -- what the next linear's fprop (row-wise) and
+ * wgrad (column-wise, token groups) consume, without reading the output back
+ * from memory.
+ *   qy_t, sy_t   : E4M3 codes [n, m] (transposed) and scales
+ *                  [ceil(m/128)][n] of y (out)
+ *   qdx_t, sdx_t : E4M3 codes [k, m] and scales [ceil(m/128)][k] of dx (out)
+ * The column groups are the 128-row (token) blocks of the output; a short
+ * last block is a short group (its amax runs over the rows present). Other
+ * arguments and errors as fp8bw_gemm_fprop_quant / fp8bw_gemm_dgrad_quant;
+ * all four extra outputs are required (non-NULL when non-empty), 16-byte
+ * aligned and must not overlap any input or each other.
+ * Source: paperlayer.ai summary, Appendix C, "FP8 implementation pipeline"
+ * (bf16 flow between the E4M3 GEMMs; the weight-gradient GEMM contracts over
+ * tokens) with the 1-D 128-groups of the arxiv-wiki summary, Approach
+ * item (4). */
+int fp8bw_gemm_fprop_quant_rowcol(const uint8_t* qx, const float* sx,
+                                  const uint8_t* qw, const float* sw,
+                                  int64_t m, int64_t n, int64_t k, uint16_t* y,
+                                  uint8_t* qy, float* sy, uint8_t* qy_t,
+                                  float* sy_t, void* stream);
+int fp8bw_gemm_dgrad_quant_rowcol(const uint8_t* qdy, const float* sdy,
+                                  const uint8_t* qw, int qw_is_transposed,
+                                  const float* sw, int64_t m, int64_t n,
+                                  int64_t k, uint16_t* dx, uint8_t* qdx,
+                                  float* sdx, uint8_t* qdx_t, float* sdx_t,
+                                  void* stream);
+
 /* ------------------------------------------------------------------------
  * Power-of-two scales on the tensor cores' block scaling.
  *

@@ -37,14 +37,14 @@ def lib():
 
 def test_every_declared_symbol_is_exported(lib):
     names = declared_functions()
-    assert len(names) == 20
+    assert len(names) == 22
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(_native.SIGNATURES)
 
 
 def test_status_strings_and_version(lib):
-    assert lib.fp8bw_version() == 105
+    assert lib.fp8bw_version() == 106
     for st in (OK, E_NULL, E_SHAPE, E_ALIGN, E_DEVICE, E_LAUNCH, E_TIMEOUT,
                E_CUDA, E_ALIAS, E_SCALE):
         s = lib.fp8bw_status_string(st).decode()

@@ -124,3 +124,42 @@ def test_gemms_write_exactly_their_outputs(m, n, k):
     rdx, rqdx, rsdx = ops.gemm_dgrad_quant(qdy, sdy, qw_t, sw)
     assert _eq(y, ry) and _eq(qy, rqy) and _eq(sy, rsy)
     assert _eq(dx, rdx) and _eq(qdx, rqdx) and _eq(sdx, rsdx)
+
+
+@pytest.mark.parametrize("m,n,k", SHAPES + [(400, 272, 256)])
+def test_newer_outputs_write_exactly_their_outputs(m, n, k):
+    """The power-of-two fp32 wgrad (store and add) and the fused row +
+    column output quantisation of fprop and dgrad."""
+    import torch
+    ops = _ops()
+    x = bf16_np_to_torch(S.bf16_normal((m, k), 0, 990, **S.X_DIST))
+    w = bf16_np_to_torch(S.bf16_normal((n, k), 0, 991, **S.W_DIST))
+    dy = bf16_np_to_torch(S.bf16_normal((m, n), 0, 992, **S.DY_DIST))
+    cd = lambda a: (a + 127) // 128  # noqa: E731
+    pqx_t, psx_t = ops.quantize_colwise(x, pow2=True)
+    pqdy_t, psdy_t = ops.quantize_colwise(dy, pow2=True)
+    qx_t, sx_t, qx, sx = ops.quantize_colwise(x, with_rowwise=True)
+    qdy_t, sdy_t, qdy, sdy = ops.quantize_colwise(dy, with_rowwise=True)
+    qw, sw, qw_t = ops.quantize_weight_block(w)
+    g = Guarded()
+    dw32, acc32 = g.make((n, k), torch.float32), g.make((n, k), torch.float32)
+    y, qy, sy = (g.make((m, n), torch.bfloat16), g.make((m, n), torch.uint8),
+                 g.make((cd(n), m), torch.float32))
+    qy_t, sy_t = g.make((n, m), torch.uint8), g.make((cd(m), n), torch.float32)
+    dx, qdx, sdx = (g.make((m, k), torch.bfloat16), g.make((m, k), torch.uint8),
+                    g.make((cd(k), m), torch.float32))
+    qdx_t, sdx_t = g.make((k, m), torch.uint8), g.make((cd(m), k), torch.float32)
+    acc32.zero_()
+    ops.fp8bw_gemm_wgrad_f32(pqdy_t, psdy_t, pqx_t, psx_t, dw32, pow2=True)
+    ops.fp8bw_gemm_wgrad_f32(pqdy_t, psdy_t, pqx_t, psx_t, acc32, accumulate=True,
+                             pow2=True)
+    ops.fp8bw_gemm_fprop_quant_rowcol(qx, sx, qw, sw, y, qy, sy, qy_t, sy_t)
+    ops.fp8bw_gemm_dgrad_quant_rowcol(qdy, sdy, qw_t, 1, sw, dx, qdx, sdx, qdx_t, sdx_t)
+    ops.fp8bw_check_device_error()
+    g.check("power-of-two fp32 wgrad and fused row + column quantisation")
+    ref32 = ops.gemm_wgrad_f32(pqdy_t, psdy_t, pqx_t, psx_t, pow2=True)
+    assert _eq(dw32, ref32) and _eq(acc32, ref32)
+    r = ops.gemm_fprop_quant_rowcol(qx, sx, qw, sw)
+    assert all(_eq(a, b) for a, b in zip((y, qy, sy, qy_t, sy_t), r))
+    r = ops.gemm_dgrad_quant_rowcol(qdy, sdy, qw_t, sw)
+    assert all(_eq(a, b) for a, b in zip((dx, qdx, sdx, qdx_t, sdx_t), r))
