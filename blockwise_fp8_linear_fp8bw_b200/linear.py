@@ -16,6 +16,10 @@ hidden flow, fp32 gradients):
                  micro-batches; the add is done by the GEMM's epilogue, for
                  either scale form), else returned in the weight's dtype.
 
+Linears that feed one another directly (BlockwiseFp8Chain) fuse the
+quantisation of every intermediate activation and gradient into the GEMM that
+produces it (row-wise and column-wise codes from the fprop / dgrad epilogue).
+
 Every step runs in the CUDA library; this module only reshapes tensors and
 keeps the codes the backward pass needs. Inputs must be bf16 CUDA tensors
 whose dimensions are multiples of 16.
@@ -102,4 +106,92 @@ class BlockwiseFp8Linear(torch.nn.Module):
             self.in_features, self.out_features, self.pow2)
 
 
-__all__ = ["BlockwiseFp8Linear", "BlockwiseFp8LinearFunction"]
+class BlockwiseFp8ChainFunction(torch.autograd.Function):
+    """y = x @ W_0.T @ W_1.T ... @ W_{L-1}.T: linears that feed one another
+    directly, each on the blockwise-FP8 path, with every intermediate
+    quantisation fused into the GEMM that produces it.
+
+    Forward: each fprop but the last also writes the row-wise (next fprop)
+    and column-wise (next wgrad) codes of its bf16 output, so the next linear
+    reads codes instead of re-reading and re-quantising the activation.
+    Backward: each dgrad but the first linear's does the same for the
+    gradient it produces, which is the previous linear's dY. The results are
+    those of the same linears run one by one (the fused codes are, bit for
+    bit, those of quantising the bf16 output)."""
+
+    @staticmethod
+    def forward(ctx, x, *weights):
+        k0 = weights[0].shape[1]
+        h = _rows(x, k0)
+        qx_t, sx_t, qx, sx = ops.quantize_colwise(h, with_rowwise=True)
+        saved = []
+        y = None
+        for i, weight in enumerate(weights):
+            w = _rows(weight, weight.shape[1])
+            qw, sw, qw_t = ops.quantize_weight_block(w, transposed=True)
+            saved += [qx_t, sx_t, qw_t, sw]
+            if i + 1 < len(weights):
+                y, qx, sx, qx_t, sx_t = ops.gemm_fprop_quant_rowcol(qx, sx, qw, sw)
+            else:
+                y = ops.gemm_fprop(qx, sx, qw, sw)
+        ctx.save_for_backward(*saved)
+        ctx.weights = weights
+        ctx.x_shape = x.shape
+        return y.reshape(*x.shape[:-1], weights[-1].shape[0])
+
+    @staticmethod
+    def backward(ctx, dy):
+        saved = ctx.saved_tensors
+        weights = ctx.weights
+        n_last = weights[-1].shape[0]
+        dy2 = _rows(dy, n_last)
+        qdy_t, sdy_t, qdy, sdy = ops.quantize_colwise(dy2, with_rowwise=True)
+        grads = [None] * len(weights)
+        dx = None
+        for i in range(len(weights) - 1, -1, -1):
+            qx_t, sx_t, qw_t, sw = saved[4 * i:4 * i + 4]
+            weight = weights[i]
+            if ctx.needs_input_grad[1 + i]:
+                main = getattr(weight, "main_grad", None)
+                if main is not None:
+                    ops.gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, main_grad=main)
+                else:
+                    dw = ops.gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t)
+                    grads[i] = dw if dw.dtype == weight.dtype else dw.to(weight.dtype)
+            if i > 0:
+                _, qdy, sdy, qdy_t, sdy_t = ops.gemm_dgrad_quant_rowcol(
+                    qdy, sdy, qw_t, sw, qw_is_transposed=True)
+            elif ctx.needs_input_grad[0]:
+                dx = ops.gemm_dgrad(qdy, sdy, qw_t, sw,
+                                    qw_is_transposed=True).reshape(ctx.x_shape)
+        return (dx, *grads)
+
+
+class BlockwiseFp8Chain(torch.nn.Module):
+    """Bias-free linears applied one after another with nothing in between
+    (features[0] -> features[1] -> ... -> features[-1]), as
+    BlockwiseFp8ChainFunction: the quantisation of every intermediate
+    activation and gradient is fused into the GEMM that produces it."""
+
+    def __init__(self, features, device=None):
+        super().__init__()
+        if len(features) < 2 or any(f % 16 for f in features):
+            raise ValueError("need at least two feature sizes, each a multiple "
+                             "of 16")
+        self.features = list(features)
+        ws = []
+        for fin, fout in zip(features[:-1], features[1:]):
+            w = torch.empty((fout, fin), dtype=torch.bfloat16, device=device)
+            torch.nn.init.normal_(w, std=0.02)
+            ws.append(torch.nn.Parameter(w))
+        self.weights = torch.nn.ParameterList(ws)
+
+    def forward(self, x):
+        return BlockwiseFp8ChainFunction.apply(x, *self.weights)
+
+    def extra_repr(self):
+        return "features=%s" % (self.features,)
+
+
+__all__ = ["BlockwiseFp8Linear", "BlockwiseFp8LinearFunction",
+           "BlockwiseFp8Chain", "BlockwiseFp8ChainFunction"]

@@ -2,7 +2,6 @@
 dX and dW (returned in the weight's dtype, or added in fp32 into
 weight.main_grad), against the oracle's quantisers and GEMMs on the same
 inputs; plus its argument checks on CPU (no CPU fallback)."""
-import numpy as np
 import pytest
 
 import oracle
@@ -50,13 +49,10 @@ def _case(pow2, main_grad, shape=(2, 144), k=400, n=528, seed=950):
     rqx_t, rsx_t = oracle.quantize_colwise(x, pow2=pow2)
     acc, bound = oracle.gemm_wgrad(rq_t, rs_t, rqx_t, rsx_t, with_bound=True)
     if main_grad:
+        # both scale forms add the fp32 dW into main_grad in the GEMM epilogue
         assert lin.weight.grad is None
         got = lin.weight.main_grad.cpu().numpy()
-        if pow2:      # the power-of-two wgrad is bf16, added into a zeroed fp32 buffer
-            bits = (got.view(np.uint32) >> 16).astype(np.uint16)
-            assert_gemm_close(bits, acc, bound, "linear dW (main_grad, pow2)")
-        else:
-            assert_gemm_close_f32(got, acc, bound, "linear dW (main_grad)")
+        assert_gemm_close_f32(got, acc, bound, "linear dW (main_grad)")
     else:
         assert lin.weight.grad.dtype == torch.bfloat16
         assert_gemm_close(torch_bf16_to_np(lin.weight.grad), acc, bound, "linear dW")
@@ -95,3 +91,68 @@ def test_library_call_from_a_fresh_thread():
     assert not err, err
     q_t, s_t, q, s = out["qs"]
     assert torch.equal(q, ref_q) and torch.equal(s.view(torch.int32), ref_s.view(torch.int32))
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("main_grad", [False, True])
+def test_chain_equals_the_linears_one_by_one(main_grad):
+    """Three linears that feed one another: the chain (quantisation of the
+    intermediate activations and gradients fused into the producing GEMMs)
+    gives, bit for bit, the output, dX and dW of the same linears run one by
+    one with their own quantisers; and the first linear's dW is within the
+    acceptance bound of the oracle's, given the gradient that reached its
+    output."""
+    import torch
+    from blockwise_fp8_linear_fp8bw_b200.linear import (BlockwiseFp8Chain,
+                                                         BlockwiseFp8Linear)
+    feats = [400, 272, 528, 144]
+    m = 288
+    chain = BlockwiseFp8Chain(feats, device="cuda")
+    singles = [BlockwiseFp8Linear(a, b, device="cuda")
+               for a, b in zip(feats[:-1], feats[1:])]
+    for i, lin in enumerate(singles):
+        w = S.bf16_normal((feats[i + 1], feats[i]), 0, 970 + i, **S.W_DIST)
+        with torch.no_grad():
+            lin.weight.copy_(bf16_np_to_torch(w))
+            chain.weights[i].copy_(bf16_np_to_torch(w))
+        if main_grad:
+            lin.weight.main_grad = torch.zeros(lin.weight.shape, dtype=torch.float32,
+                                               device="cuda")
+            chain.weights[i].main_grad = torch.zeros(lin.weight.shape,
+                                                     dtype=torch.float32, device="cuda")
+    x = S.bf16_normal((m, feats[0]), 0, 975, **S.X_DIST)
+    dy = S.bf16_normal((m, feats[-1]), 0, 976, **S.DY_DIST)
+    xa = bf16_np_to_torch(x).requires_grad_(True)
+    xb = bf16_np_to_torch(x).requires_grad_(True)
+    g = bf16_np_to_torch(dy)
+    ya = chain(xa)
+    ya.backward(g)
+    outs = []
+    h = xb
+    for lin in singles:
+        h = lin(h)
+        outs.append(h)
+    seen = {}
+    outs[0].register_hook(lambda t: seen.setdefault("dy0", t.detach().clone()))
+    outs[-1].backward(g)
+    torch.cuda.synchronize()
+
+    eq = lambda a, b: torch.equal(a.view(torch.int16), b.view(torch.int16))  # noqa: E731
+    assert eq(ya, outs[-1]) and eq(xa.grad, xb.grad)
+    for i, lin in enumerate(singles):
+        if main_grad:
+            assert chain.weights[i].grad is None
+            assert torch.equal(chain.weights[i].main_grad.view(torch.int32),
+                               lin.weight.main_grad.view(torch.int32))
+        else:
+            assert eq(chain.weights[i].grad, lin.weight.grad)
+
+    rq_t, rs_t = oracle.quantize_colwise(torch_bf16_to_np(seen["dy0"]))
+    rqx_t, rsx_t = oracle.quantize_colwise(x)
+    acc, bound = oracle.gemm_wgrad(rq_t, rs_t, rqx_t, rsx_t, with_bound=True)
+    if main_grad:
+        assert_gemm_close_f32(chain.weights[0].main_grad.cpu().numpy(), acc, bound,
+                              "chain dW_0 (main_grad)")
+    else:
+        assert_gemm_close(torch_bf16_to_np(chain.weights[0].grad), acc, bound,
+                          "chain dW_0")
