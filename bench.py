@@ -463,6 +463,49 @@ def time_next_rows(o, bufs, stream, warmup, rounds):
                 "timed after the step" % (names, TOKENS)}
     del qy, sy, qdx, sdx
 
+    # ... and writing both the row-wise and the transposed column-wise codes
+    # (all a consumer linear needs), against the GEMMs followed by the
+    # one-pass row + column quantiser.
+    fused, unfused = [], []
+    for b in bufs:
+        m = TOKENS
+        u8, f32 = torch.uint8, torch.float32
+        cd = lambda a: (a + 127) // 128  # noqa: E731
+        qy, sy = (torch.empty((m, b.n), dtype=u8, device=dev),
+                  torch.empty((cd(b.n), m), dtype=f32, device=dev))
+        qy_t, sy_t = (torch.empty((b.n, m), dtype=u8, device=dev),
+                      torch.empty((cd(m), b.n), dtype=f32, device=dev))
+        qdx, sdx = (torch.empty((m, b.k), dtype=u8, device=dev),
+                    torch.empty((cd(b.k), m), dtype=f32, device=dev))
+        qdx_t, sdx_t = (torch.empty((b.k, m), dtype=u8, device=dev),
+                        torch.empty((cd(m), b.k), dtype=f32, device=dev))
+        fused += [
+            (lambda b=b, o4=(qy, sy, qy_t, sy_t): o.fp8bw_gemm_fprop_quant_rowcol(
+                b.qx, b.sx, b.qw, b.sw, b.y, *o4, stream)),
+            (lambda b=b, o4=(qdx, sdx, qdx_t, sdx_t): o.fp8bw_gemm_dgrad_quant_rowcol(
+                b.qdy, b.sdy, b.qw_t, 1, b.sw, b.dx, *o4, stream))]
+        unfused += [
+            (lambda b=b: o.fp8bw_gemm_fprop(b.qx, b.sx, b.qw, b.sw, b.y,
+                                            stream)),
+            (lambda b=b, o4=(qy_t, sy_t, qy, sy): o.fp8bw_quantize_colwise(
+                b.y, *o4, stream)),
+            (lambda b=b: o.fp8bw_gemm_dgrad(b.qdy, b.sdy, b.qw_t, 1, b.sw,
+                                            b.dx, stream)),
+            (lambda b=b, o4=(qdx_t, sdx_t, qdx, sdx): o.fp8bw_quantize_colwise(
+                b.dx, *o4, stream))]
+    t_f = seq_time(fused)
+    t_u = seq_time(unfused)
+    out["gemm_fused_rowcol_quant"] = {
+        "achieved": gfl / (t_f * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "ms_fused": t_f, "ms_gemm_then_quantiser": t_u,
+        "saved_frac": 1.0 - t_f / t_u,
+        "what": "fprop and dgrad of the %s linears (M=%d) writing bf16 "
+                "plus the row-wise and the transposed column-wise E4M3 codes "
+                "and scales of that output, against the same GEMMs followed "
+                "by the one-pass row + column quantiser; timed after the "
+                "step" % (names, TOKENS)}
+    del fused, unfused
+
     # The whole step again with power-of-two scales (quantisers and GEMMs on
     # the tensor cores' UE8M0 block scaling), same buffers and order.
     step = []

@@ -103,13 +103,17 @@ def test_next_rows_host_logic_with_stubbed_device(monkeypatch):
     bufs = [_FakeLinear("gate_up", 128, 256), _FakeLinear("down", 256, 128)]
     out = bench.time_next_rows(lib, bufs, None, 3, 5)
     assert set(out) == {"wgrad_f32_accumulate", "gemm_fused_rowwise_quant",
-                        "pow2_step"}
+                        "gemm_fused_rowcol_quant", "pow2_step"}
     assert "gate/up and down linears" in out["wgrad_f32_accumulate"]["what"]
     assert "gate/up and down linears" in out["gemm_fused_rowwise_quant"]["what"]
+    assert "gate/up and down linears" in out["gemm_fused_rowcol_quant"]["what"]
+    assert lib.calls["fp8bw_gemm_fprop_quant_rowcol"] == \
+        lib.calls["fp8bw_gemm_dgrad_quant_rowcol"]
     assert ("%d-layer" % bench.LAYERS) in out["pow2_step"]["what"]
     assert out["wgrad_f32_accumulate"]["launches"] == 5 * len(bufs)
     assert lib.calls["fp8bw_gemm_wgrad_f32"] == 2 * (3 + 5)
-    assert lib.calls["fp8bw_gemm_fprop_quant"] == lib.calls["fp8bw_gemm_fprop"]
+    # fprop runs in the row-wise and the row + column comparison alike
+    assert 2 * lib.calls["fp8bw_gemm_fprop_quant"] == lib.calls["fp8bw_gemm_fprop"]
     assert set(out["pow2_step"]["breakdown"]) == {
         "quant_weight_block", "quant_rowcol", "gemm_block_scaled",
         "gemm_vector_scaled"}
