@@ -261,7 +261,9 @@ int launch_gemm_pair(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t s
   g.st_out = p.st_out;
   const int64_t tiles = static_cast<int64_t>(g.tiles_m) * g.tiles_n;
   const int clusters = static_cast<int>(std::min<int64_t>(tiles, max_clusters));
-  kernel<<<2 * clusters, gemm::kThreads, L::kAlloc, stream>>>(tm_a, tm_b, tm_out, g);
+  if (launch_kernel(kernel, dim3(2 * clusters), dim3(gemm::kThreads), L::kAlloc, stream, tm_a,
+                    tm_b, tm_out, g) != cudaSuccess)
+    return FP8BW_ERR_LAUNCH;
   return cudaGetLastError() == cudaSuccess ? FP8BW_OK : FP8BW_ERR_LAUNCH;
 }
 
@@ -311,7 +313,9 @@ int launch_gemm_pow2(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t s
   g.nblk = static_cast<int>(cdiv(p.no, 128));
   const int64_t tiles = static_cast<int64_t>(g.tiles_m) * g.tiles_n;
   const int clusters = static_cast<int>(std::min<int64_t>(tiles, max_clusters));
-  kernel<<<2 * clusters, gemm_pow2::kThreads, L::kAlloc, stream>>>(tm_a, tm_b, tm_out, g);
+  if (launch_kernel(kernel, dim3(2 * clusters), dim3(gemm_pow2::kThreads), L::kAlloc, stream,
+                    tm_a, tm_b, tm_out, g) != cudaSuccess)
+    return FP8BW_ERR_LAUNCH;
   return cudaGetLastError() == cudaSuccess ? FP8BW_OK : FP8BW_ERR_LAUNCH;
 }
 

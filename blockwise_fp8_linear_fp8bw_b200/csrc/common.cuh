@@ -52,6 +52,50 @@ int prepare_for_device(DevicePrep& p, int dev, int* value, Fn&& fn) {
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch. Every kernel of the library is launched with
+// programmatic stream serialisation: it may be scheduled while the kernel
+// before it in the stream is still running, does its set-up (barriers, TMEM,
+// tensor-map prefetch; nothing that reads or writes global memory), and
+// then waits in grid_dependency_wait() until that kernel has completed and
+// its memory operations are visible, before its first global access. It
+// lets the kernel after it be scheduled the same way (launch_dependents()),
+// so launch latency and set-up overlap the previous kernel's last wave.
+// Without the launch attribute both instructions do nothing.
+// ---------------------------------------------------------------------------
+#ifndef FP8BW_PDL
+#define FP8BW_PDL 1
+#endif
+
+__device__ __forceinline__ void grid_dependency_wait() {
+#if FP8BW_PDL
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+#endif
+}
+
+__device__ __forceinline__ void launch_dependents() {
+#if FP8BW_PDL
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+#endif
+}
+
+// Launch `kernel` on `stream` with programmatic stream serialisation.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = FP8BW_PDL ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// ---------------------------------------------------------------------------
 // Output modes of the GEMM epilogues.
 // ---------------------------------------------------------------------------
 constexpr int kOutBf16 = 0;       // bf16 store

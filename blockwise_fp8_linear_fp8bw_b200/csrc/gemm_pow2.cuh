@@ -165,6 +165,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Set-up done: let the next kernel be scheduled, and wait for the previous
+  // one before any global memory is read or written.
+  launch_dependents();
+  grid_dependency_wait();
 
   const int num_tiles = g.tiles_m * g.tiles_n;
   const int C = g.chunks;

@@ -120,6 +120,10 @@ __global__ void __launch_bounds__(kQThreads, 2)
     prefetch_tmap(&tm_x);
   }
   __syncthreads();
+  // Set-up done: let the next kernel be scheduled, and wait for the previous
+  // one before any global memory is read or written.
+  launch_dependents();
+  grid_dependency_wait();
   // Thread 0 keeps, per input buffer, the phase parity of a load it issued and
   // that nobody has waited for yet (-1: none).
   int pend[2] = {-1, -1};
@@ -367,7 +371,9 @@ int launch_quantize(int mode, bool pow2, const uint16_t* x, int64_t rows, int64_
   });
   if (pst != FP8BW_OK) return pst;
   const Kernel kernel = kernels[(mode >= 0 && mode < 4 ? mode : kModeBlock) + (pow2 ? 4 : 0)];
-  kernel<<<grid, kQThreads, QuantSmem::kAlloc, stream>>>(tm, a);
+  if (launch_kernel(kernel, dim3(grid), dim3(kQThreads), QuantSmem::kAlloc, stream, tm, a) !=
+      cudaSuccess)
+    return FP8BW_ERR_LAUNCH;
   return cudaGetLastError() == cudaSuccess ? FP8BW_OK : FP8BW_ERR_LAUNCH;
 }
 
