@@ -5,13 +5,14 @@ One step = the whole hot path over the linear stack of one 28-layer
 Qwen3-1.7B-shaped training step at M = 16384 tokens (4 x 4096): for every
 layer and each of its four linears (QKV 2048->4096, O 2048->2048, gate/up
 2048->12288, down 6144->2048):
-  1. 128x128 block quantisation of W (codes + transposed codes + scales)
+  1. 128x128 block quantisation of W (codes + transposed codes + scales;
+     the four weights of a layer in one launch)
   2. row-wise + column-wise 1x128 / 128x1 quantisation of X (one pass)
   3. fprop  Y  = X W^T
   4. row-wise + column-wise quantisation of dY (one pass)
   5. dgrad  dX = dY W
   6. wgrad  dW = dY^T X
-= 672 kernel launches, 138.5 TFLOP of GEMM work per step.
+= 588 kernel launches (28 x (1 + 4 x 5)), 138.5 TFLOP of GEMM work per step.
 
 Inputs are seeded synthetic tensors (synthetic/): X ~ N(0,1) with 0.1% x50
 outliers, W ~ N(0,0.02), dY ~ N(0,1e-3) with 0.1% x100 outliers. Every layer
@@ -328,20 +329,24 @@ class LinearBuffers:
         self.qdy_t, self.sdy_t = e((n, m), u8), e((cd(m), n), f32)
         self.y, self.dx, self.dw = e((m, n), bf), e((m, k), bf), e((n, k), bf)
 
+    def weight_bytes(self):
+        """Algorithmic bytes of this weight's block quantisation (bf16 in,
+        codes, transposed codes, scales)."""
+        n, k = self.n, self.k
+        cd = lambda a: (a + 127) // 128  # noqa: E731
+        return n * k * 2 + 2 * n * k + 4 * cd(n) * cd(k)
+
     def ops(self, o, stream, pow2=False):
-        """[(kernel kind, algorithmic units, callable)] of this linear; pow2
-        selects the power-of-two-scale quantisers and GEMMs."""
+        """[(kernel kind, algorithmic units, callable)] of this linear after
+        its weight is quantised (layer_ops quantises a layer's weights in one
+        launch); pow2 selects the power-of-two-scale quantisers and GEMMs."""
         m, k, n = TOKENS, self.k, self.n
         cd = lambda a: (a + 127) // 128  # noqa: E731
-        wq_bytes = n * k * 2 + 2 * n * k + 4 * cd(n) * cd(k)
         xq_bytes = m * k * 2 + 2 * m * k + 4 * (m * cd(k) + cd(m) * k)
         dyq_bytes = m * n * 2 + 2 * m * n + 4 * (m * cd(n) + cd(m) * n)
         f = 2 * m * n * k
         p2 = pow2
         return [
-            ("quant_weight_block", wq_bytes,
-             lambda: o.fp8bw_quantize_weight_block(self.w, self.qw, self.sw,
-                                                   self.qw_t, stream, pow2=p2)),
             ("quant_rowcol", xq_bytes,
              lambda: o.fp8bw_quantize_colwise(self.x, self.qx_t, self.sx_t,
                                               self.qx, self.sx, stream,
@@ -360,6 +365,20 @@ class LinearBuffers:
              lambda: o.fp8bw_gemm_wgrad(self.qdy_t, self.sdy_t, self.qx_t,
                                         self.sx_t, self.dw, stream, pow2=p2)),
         ]
+
+
+def layer_ops(bufs, o, stream, pow2=False):
+    """The ops of one layer: its weights' 128x128 block quantisation in one
+    launch (all weights are quantised once per step, before they are used),
+    then each linear's quantisers and GEMMs."""
+    ws = [b.w for b in bufs]
+    qs, ss, qts = [b.qw for b in bufs], [b.sw for b in bufs], [b.qw_t for b in bufs]
+    out = [("quant_weight_block", sum(b.weight_bytes() for b in bufs),
+            lambda: o.fp8bw_quantize_weight_block_batch(ws, qs, ss, qts, stream,
+                                                        pow2=pow2))]
+    for b in bufs:
+        out.extend(b.ops(o, stream, pow2=pow2))
+    return out
 
 
 def linear_names(kinds):
@@ -510,8 +529,7 @@ def time_next_rows(o, bufs, stream, warmup, rounds):
     # the tensor cores' UE8M0 block scaling), same buffers and order.
     step = []
     for _layer in range(LAYERS):
-        for b in bufs:
-            step.extend(b.ops(o, stream, pow2=True))
+        step.extend(layer_ops(bufs, o, stream, pow2=True))
     with torch.cuda.stream(stream):
         for _ in range(warmup):
             for _, _, fn in step:
@@ -644,8 +662,7 @@ def measure_replica(args, world, local):
     bufs = [LinearBuffers(kind, k, n, dev) for kind, k, n in kinds()]
     step_ops = []
     for _layer in range(LAYERS):
-        for b in bufs:
-            step_ops.extend(b.ops(o, stream))
+        step_ops.extend(layer_ops(bufs, o, stream))
     flops = step_gemm_flops()
     assert flops == sum(u for kk, u, _ in step_ops if kk.startswith("gemm"))
 
@@ -754,12 +771,13 @@ def measure_replica(args, world, local):
                     if used[sl][i]:
                         stream.wait_event(fetched[sl][i])
                     b.x, b.w, b.dy, b.dw = dx_, dw_, ddy, ddw
-                    for _, _, fn in b.ops(o, stream):
-                        fn()
+                for _, _, fn in layer_ops(bufs, o, stream):
+                    fn()
+                for i, (b, (hx, hw, hdy, hdw)) in enumerate(zip(bufs, pinned)):
                     computed[sl][i].record(stream)
                     with torch.cuda.stream(down):
                         down.wait_event(computed[sl][i])
-                        hdw.copy_(ddw, non_blocking=True)
+                        hdw.copy_(b.dw, non_blocking=True)
                         fetched[sl][i].record(down)
                     used[sl][i] = True
 
@@ -799,9 +817,9 @@ def measure_replica(args, world, local):
         e2e = {"value": weak_scaling_value(world, flops, e2e_ms * 1e-3) / 1e12,
                "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-               "copies": "per layer, X/W/dY uploaded from pinned host memory "
-                         "on a copy stream while the previous layer computes; "
-                         "dW downloaded on another stream"}
+               "copies": "per layer, X/W/dY of its linears uploaded from pinned "
+                         "host memory on a copy stream while the previous layer "
+                         "computes; dW downloaded on another stream"}
 
     return {"ms": ms, "flops": flops, "per_kind": per_kind,
             "next_rows": next_rows, "clocks": clk, "e2e": e2e,

@@ -12,11 +12,18 @@ _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
 _INT = ctypes.c_int
 
+class WeightBlockJob(ctypes.Structure):
+    """fp8bw_weight_block_job of include/fp8bw.h."""
+    _fields_ = [("w", _P), ("n", _I64), ("k", _I64), ("q", _P), ("s", _P),
+                ("q_t", _P)]
+
+
 # name -> (argtypes, restype), in the order of include/fp8bw.h
 SIGNATURES = {
     "fp8bw_quantize_rowwise": ([_P, _I64, _I64, _P, _P, _P], _INT),
     "fp8bw_quantize_colwise": ([_P, _I64, _I64, _P, _P, _P, _P, _P], _INT),
     "fp8bw_quantize_weight_block": ([_P, _I64, _I64, _P, _P, _P, _P], _INT),
+    "fp8bw_quantize_weight_block_batch": ([_P, _INT, _P], _INT),
     "fp8bw_gemm_fprop": ([_P, _P, _P, _P, _I64, _I64, _I64, _P, _P], _INT),
     "fp8bw_gemm_dgrad": ([_P, _P, _P, _INT, _P, _I64, _I64, _I64, _P, _P],
                          _INT),
@@ -34,6 +41,7 @@ SIGNATURES = {
     "fp8bw_quantize_rowwise_pow2": ([_P, _I64, _I64, _P, _P, _P], _INT),
     "fp8bw_quantize_colwise_pow2": ([_P, _I64, _I64, _P, _P, _P, _P, _P], _INT),
     "fp8bw_quantize_weight_block_pow2": ([_P, _I64, _I64, _P, _P, _P, _P], _INT),
+    "fp8bw_quantize_weight_block_batch_pow2": ([_P, _INT, _P], _INT),
     "fp8bw_gemm_fprop_pow2": ([_P, _P, _P, _P, _I64, _I64, _I64, _P, _P], _INT),
     "fp8bw_gemm_dgrad_pow2": ([_P, _P, _P, _INT, _P, _I64, _I64, _I64, _P,
                                _P], _INT),

@@ -391,7 +391,7 @@ using namespace fp8bw;
 
 extern "C" {
 
-int fp8bw_version(void) { return 106; }
+int fp8bw_version(void) { return 107; }
 
 const char* fp8bw_status_string(int status) {
   switch (status) {
@@ -459,8 +459,10 @@ int quantize_colwise(bool pow2, const uint16_t* x, int64_t rows, int64_t cols, u
                          static_cast<cudaStream_t>(stream));
 }
 
-int quantize_weight_block(bool pow2, const uint16_t* w, int64_t n, int64_t k, uint8_t* q,
-                          float* s, uint8_t* q_t, void* stream) {
+// Argument checks of one 128x128 block quantisation (shape, NULL, alignment,
+// outputs against its own input).
+int weight_block_args_status(const uint16_t* w, int64_t n, int64_t k, const uint8_t* q,
+                             const float* s, const uint8_t* q_t) {
   if (!dim_ok(n) || !dim_ok(k) || cdiv(n, 128) > 65535 ||
       cdiv(n, 128) * cdiv(k, 128) > INT32_MAX)
     return FP8BW_ERR_SHAPE;
@@ -471,6 +473,13 @@ int quantize_weight_block(bool pow2, const uint16_t* w, int64_t n, int64_t k, ui
   if (overlap(rw, range_of(q, n * k)) || overlap(rw, range_of(s, cdiv(n, 128) * cdiv(k, 128) * 4)) ||
       (q_t && overlap(rw, range_of(q_t, n * k))))
     return FP8BW_ERR_ALIAS;
+  return FP8BW_OK;
+}
+
+int quantize_weight_block(bool pow2, const uint16_t* w, int64_t n, int64_t k, uint8_t* q,
+                          float* s, uint8_t* q_t, void* stream) {
+  const int ast = weight_block_args_status(w, n, k, q, s, q_t);
+  if (ast != FP8BW_OK) return ast;
   DeviceInfo dev;
   int st = current_device_info(&dev);
   if (st != FP8BW_OK) return st;
@@ -479,9 +488,53 @@ int quantize_weight_block(bool pow2, const uint16_t* w, int64_t n, int64_t k, ui
                          static_cast<cudaStream_t>(stream));
 }
 
+int quantize_weight_block_batch(bool pow2, const fp8bw_weight_block_job* jobs, int count,
+                                void* stream) {
+  if (count < 0 || count > kMaxQuantJobs) return FP8BW_ERR_SHAPE;
+  if (count > 0 && jobs == nullptr) return FP8BW_ERR_NULL;
+  Range ins[kMaxQuantJobs], outs[3 * kMaxQuantJobs];
+  int nout = 0;
+  QuantJob qj[kMaxQuantJobs];
+  int nj = 0;
+  for (int i = 0; i < count; ++i) {
+    const fp8bw_weight_block_job& j = jobs[i];
+    const int st = weight_block_args_status(j.w, j.n, j.k, j.q, j.s, j.q_t);
+    if (st != FP8BW_OK) return st;
+    ins[i] = range_of(j.w, j.n * j.k * 2);
+    outs[nout++] = range_of(j.q, j.n * j.k);
+    outs[nout++] = range_of(j.s, cdiv(j.n, 128) * cdiv(j.k, 128) * 4);
+    outs[nout++] = range_of(j.q_t, j.q_t ? j.n * j.k : 0);
+    if (j.n > 0 && j.k > 0)   // an empty weight is a no-op
+      qj[nj++] = QuantJob{j.w, j.n, j.k, j.q, nullptr, j.q_t, nullptr, j.s};
+  }
+  // no output may overlap any job's input or another output
+  for (int o = 0; o < nout; ++o) {
+    for (int i = 0; i < count; ++i)
+      if (overlap(outs[o], ins[i])) return FP8BW_ERR_ALIAS;
+    for (int o2 = o + 1; o2 < nout; ++o2)
+      if (overlap(outs[o], outs[o2])) return FP8BW_ERR_ALIAS;
+  }
+  DeviceInfo dev;
+  int st = current_device_info(&dev);
+  if (st != FP8BW_OK) return st;
+  if (nj == 0) return FP8BW_OK;
+  return launch_quantize_jobs(kModeBlock, pow2, qj, nj, dev.ordinal, dev.sm_count,
+                              static_cast<cudaStream_t>(stream));
+}
+
 }  // namespace
 
 extern "C" {
+
+int fp8bw_quantize_weight_block_batch(const fp8bw_weight_block_job* jobs, int count,
+                                      void* stream) {
+  return quantize_weight_block_batch(false, jobs, count, stream);
+}
+
+int fp8bw_quantize_weight_block_batch_pow2(const fp8bw_weight_block_job* jobs, int count,
+                                           void* stream) {
+  return quantize_weight_block_batch(true, jobs, count, stream);
+}
 
 int fp8bw_quantize_rowwise(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* q, float* s,
                            void* stream) {

@@ -32,6 +32,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
+#include <cstring>
+
 #include "common.cuh"
 
 namespace fp8bw {
@@ -57,6 +59,19 @@ struct QuantArgs {
   uint8_t* q_col;   // [cols, rows]  (block mode: q_t, may be null)
   float* s_col;     // [ceil(rows/128)][cols]
   float* s_block;   // [ceil(rows/128)][ceil(cols/128)]
+};
+
+// One launch quantises up to kMaxQuantJobs tensors ("jobs") in the same mode:
+// their 128x128 tiles are numbered one after another (job j owns tiles
+// [tile_end[j-1], tile_end[j])) and the persistent CTAs walk the combined
+// range, so small tensors share one launch's ramp and tail.
+constexpr int kMaxQuantJobs = 8;
+
+struct QuantJobs {
+  CUtensorMap maps[kMaxQuantJobs];   // bf16 input of each job
+  QuantArgs args[kMaxQuantJobs];
+  int tile_end[kMaxQuantJobs];       // cumulative tile counts
+  int count;
 };
 
 struct QuantSmem {
@@ -90,7 +105,7 @@ __device__ __forceinline__ int t_unit_offset(int k, int u) {
 
 template <int MODE, bool POW2>
 __global__ void __launch_bounds__(kQThreads, 2)
-    quant_tile_kernel(const __grid_constant__ CUtensorMap tm_x, const QuantArgs a) {
+    quant_tile_kernel(const __grid_constant__ QuantJobs jobs) {
   extern __shared__ uint8_t qsmem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(qsmem_raw) + 127) & ~static_cast<uintptr_t>(127));
@@ -109,15 +124,29 @@ __global__ void __launch_bounds__(kQThreads, 2)
   const int lane = t & 31;
   const int rb = t >> 4;   // 0..15: rows 8*rb .. 8*rb+7 of the tile
   const int cg = t & 15;   // 0..15: columns 8*cg .. 8*cg+7 of the tile
-  const int64_t rows = a.rows, cols = a.cols;
-  const int num_tiles = a.tiles_r * a.tiles_c;
+  const int num_tiles = jobs.tile_end[jobs.count - 1];
+  // The job that owns combined tile `tile`.
+  auto job_of = [&](int tile) {
+    int j = 0;
+    while (j + 1 < jobs.count && tile >= jobs.tile_end[j]) ++j;
+    return j;
+  };
+  // TMA load of combined tile `tile` into input buffer `b`.
+  auto load_tile = [&](int tile, int b) {
+    const int j = job_of(tile);
+    const int lt = tile - (j > 0 ? jobs.tile_end[j - 1] : 0);
+    const int tcs = jobs.args[j].tiles_c;
+    mbar_arrive_expect_tx(bar0 + 8u * b, kQTileBytes);
+    tma_load_2d(sbase + S::kIn + b * kQTileBytes, &jobs.maps[j], bar0 + 8u * b,
+                (lt % tcs) * kQTile, (lt / tcs) * kQTile);
+  };
 
   if (t == 0) {
     mbar_init(bar0, 1);
     mbar_init(bar0 + 8, 1);
     *abort_flag = 0u;
     fence_mbar_init();
-    prefetch_tmap(&tm_x);
+    for (int j = 0; j < jobs.count; ++j) prefetch_tmap(&jobs.maps[j]);
   }
   __syncthreads();
   // Set-up done: let the next kernel be scheduled, and wait for the previous
@@ -131,9 +160,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
     for (int k = 0; k < 2; ++k) {
       const int tile = blockIdx.x + k * gridDim.x;
       if (tile < num_tiles) {
-        mbar_arrive_expect_tx(bar0 + 8u * k, kQTileBytes);
-        tma_load_2d(sbase + S::kIn + k * kQTileBytes, &tm_x, bar0 + 8u * k,
-                    (tile % a.tiles_c) * kQTile, (tile / a.tiles_c) * kQTile);
+        load_tile(tile, k);
         pend[k] = 0;
       }
     }
@@ -145,7 +172,11 @@ __global__ void __launch_bounds__(kQThreads, 2)
     const bool got = mbar_wait(bar0 + 8u * buf, (k >> 1) & 1, abort_flag, kErrTimeoutTma);
     if (!__syncthreads_and(got ? 1 : 0)) break;
     pend[buf] = -1;
-    const int tr = tile / a.tiles_c, tc = tile % a.tiles_c;
+    const int job = job_of(tile);
+    const QuantArgs& a = jobs.args[job];
+    const int64_t rows = a.rows, cols = a.cols;
+    const int lt = tile - (job > 0 ? jobs.tile_end[job - 1] : 0);
+    const int tr = lt / a.tiles_c, tc = lt % a.tiles_c;
     const int64_t r0 = static_cast<int64_t>(tr) * kQTile + rb * 8;
     const int64_t c0 = static_cast<int64_t>(tc) * kQTile + cg * 8;
     // rows and cols are multiples of 16: an 8-wide run is all in or all out.
@@ -169,9 +200,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
     if (t == 0) {
       const int next = tile + 2 * gridDim.x;
       if (next < num_tiles) {
-        mbar_arrive_expect_tx(bar0 + 8u * buf, kQTileBytes);
-        tma_load_2d(sbase + S::kIn + buf * kQTileBytes, &tm_x, bar0 + 8u * buf,
-                    (next % a.tiles_c) * kQTile, (next / a.tiles_c) * kQTile);
+        load_tile(next, buf);
         pend[buf] = ((k >> 1) + 1) & 1;
       }
     }
@@ -343,18 +372,41 @@ __global__ void __launch_bounds__(kQThreads, 2)
 // swizzle); out-of-range elements read as zero.
 int encode_bf16_in(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows);
 
-// Launchers (shapes and pointers already validated by the C ABI layer).
-int launch_quantize(int mode, bool pow2, const uint16_t* x, int64_t rows, int64_t cols,
-                    uint8_t* q_row, float* s_row, uint8_t* q_col, float* s_col, float* s_block,
-                    int device, int sm_count, cudaStream_t stream) {
-  QuantArgs a{rows, cols, static_cast<int>((rows + kQTile - 1) / kQTile),
-              static_cast<int>((cols + kQTile - 1) / kQTile), q_row, s_row, q_col, s_col, s_block};
-  CUtensorMap tm;
-  const int st = encode_bf16_in(&tm, x, static_cast<uint64_t>(cols), static_cast<uint64_t>(rows));
-  if (st != FP8BW_OK) return st;
-  const int tiles = a.tiles_r * a.tiles_c;
-  const int grid = tiles < 2 * sm_count ? tiles : 2 * sm_count;
-  using Kernel = void (*)(CUtensorMap, QuantArgs);
+// One quantisation job of a launch (shapes and pointers already validated
+// by the C ABI layer).
+struct QuantJob {
+  const uint16_t* x;
+  int64_t rows, cols;
+  uint8_t* q_row;
+  float* s_row;
+  uint8_t* q_col;
+  float* s_col;
+  float* s_block;
+};
+
+// Launch one kernel over 1..kMaxQuantJobs jobs of the same mode.
+int launch_quantize_jobs(int mode, bool pow2, const QuantJob* jb, int count, int device,
+                         int sm_count, cudaStream_t stream) {
+  if (count < 1 || count > kMaxQuantJobs) return FP8BW_ERR_SHAPE;
+  QuantJobs jobs;
+  memset(&jobs, 0, sizeof jobs);
+  int64_t tiles = 0;
+  for (int i = 0; i < count; ++i) {
+    QuantArgs& a = jobs.args[i];
+    a = QuantArgs{jb[i].rows, jb[i].cols, static_cast<int>((jb[i].rows + kQTile - 1) / kQTile),
+                  static_cast<int>((jb[i].cols + kQTile - 1) / kQTile), jb[i].q_row, jb[i].s_row,
+                  jb[i].q_col, jb[i].s_col, jb[i].s_block};
+    const int st = encode_bf16_in(&jobs.maps[i], jb[i].x, static_cast<uint64_t>(jb[i].cols),
+                                  static_cast<uint64_t>(jb[i].rows));
+    if (st != FP8BW_OK) return st;
+    tiles += static_cast<int64_t>(a.tiles_r) * a.tiles_c;
+    if (tiles > INT32_MAX) return FP8BW_ERR_SHAPE;
+    jobs.tile_end[i] = static_cast<int>(tiles);
+  }
+  jobs.count = count;
+  if (tiles == 0) return FP8BW_OK;
+  const int grid = static_cast<int>(tiles < 2 * sm_count ? tiles : 2 * sm_count);
+  using Kernel = void (*)(QuantJobs);
   static const Kernel kernels[8] = {
       quant_tile_kernel<kModeRow, false>,    quant_tile_kernel<kModeCol, false>,
       quant_tile_kernel<kModeRowCol, false>, quant_tile_kernel<kModeBlock, false>,
@@ -371,10 +423,18 @@ int launch_quantize(int mode, bool pow2, const uint16_t* x, int64_t rows, int64_
   });
   if (pst != FP8BW_OK) return pst;
   const Kernel kernel = kernels[(mode >= 0 && mode < 4 ? mode : kModeBlock) + (pow2 ? 4 : 0)];
-  if (launch_kernel(kernel, dim3(grid), dim3(kQThreads), QuantSmem::kAlloc, stream, tm, a) !=
+  if (launch_kernel(kernel, dim3(grid), dim3(kQThreads), QuantSmem::kAlloc, stream, jobs) !=
       cudaSuccess)
     return FP8BW_ERR_LAUNCH;
   return cudaGetLastError() == cudaSuccess ? FP8BW_OK : FP8BW_ERR_LAUNCH;
+}
+
+// Launch for one tensor.
+int launch_quantize(int mode, bool pow2, const uint16_t* x, int64_t rows, int64_t cols,
+                    uint8_t* q_row, float* s_row, uint8_t* q_col, float* s_col, float* s_block,
+                    int device, int sm_count, cudaStream_t stream) {
+  const QuantJob job{x, rows, cols, q_row, s_row, q_col, s_col, s_block};
+  return launch_quantize_jobs(mode, pow2, &job, 1, device, sm_count, stream);
 }
 
 }  // namespace fp8bw

@@ -5,6 +5,8 @@ current CUDA stream -> cudaStream_t); every step of the computation runs in
 the CUDA library. The `fp8bw_*` functions take pre-allocated outputs; the
 short-named helpers allocate the outputs with torch and call them.
 """
+import ctypes
+
 import torch
 
 from . import _native
@@ -139,6 +141,32 @@ def fp8bw_quantize_weight_block(w, q, s, q_t=None, stream=None,
         _expect(q_t, torch.uint8, (k, n), "q_t")
     _call(_fn('fp8bw_quantize_weight_block', pow2), (w, q, s, q_t), stream,
           _ptr(w), n, k, _ptr(q), _ptr(s), _ptr(q_t))
+
+
+def fp8bw_quantize_weight_block_batch(ws, qs, ss, q_ts=None, stream=None,
+                                      pow2=False):
+    """Block quantisation of up to 8 weights in one launch: job i is
+    fp8bw_quantize_weight_block(ws[i], qs[i], ss[i], q_ts[i])."""
+    count = len(ws)
+    if q_ts is None:
+        q_ts = [None] * count
+    if not (len(qs) == len(ss) == len(q_ts) == count):
+        raise ValueError("ws, qs, ss and q_ts must have one entry per weight")
+    if count == 0:
+        return
+    jobs = (_native.WeightBlockJob * count)()
+    tensors = []
+    for i, (w, q, s, q_t) in enumerate(zip(ws, qs, ss, q_ts)):
+        n, k = w.shape
+        _expect(w, torch.bfloat16, (n, k), "ws[%d]" % i)
+        _expect(q, torch.uint8, (n, k), "qs[%d]" % i)
+        _expect(s, torch.float32, (_cdiv(n, 128), _cdiv(k, 128)), "ss[%d]" % i)
+        if q_t is not None:
+            _expect(q_t, torch.uint8, (k, n), "q_ts[%d]" % i)
+        jobs[i] = _native.WeightBlockJob(_ptr(w), n, k, _ptr(q), _ptr(s), _ptr(q_t))
+        tensors += [w, q, s, q_t]
+    _call(_fn("fp8bw_quantize_weight_block_batch", pow2), tensors, stream,
+          ctypes.cast(jobs, ctypes.c_void_p), count)
 
 
 def fp8bw_gemm_fprop(qx, sx, qw, sw, y, stream=None, pow2=False):
@@ -425,3 +453,19 @@ def gemm_dgrad_quant_rowcol(qdy, sdy, qw, sw, qw_is_transposed=True,
     fp8bw_gemm_dgrad_quant_rowcol(qdy, sdy, qw, qw_is_transposed, sw, dx, qdx,
                                   sdx, qdx_t, sdx_t, stream)
     return dx, qdx, sdx, qdx_t, sdx_t
+
+
+def quantize_weight_block_batch(ws, transposed=True, stream=None, pow2=False):
+    """-> [(q, s, q_t)] for each weight, all quantised in one launch."""
+    out = []
+    for w in ws:
+        n, k = w.shape
+        dev = w.device
+        out.append((torch.empty((n, k), dtype=torch.uint8, device=dev),
+                    torch.empty((_cdiv(n, 128), _cdiv(k, 128)), dtype=torch.float32,
+                                device=dev),
+                    torch.empty((k, n), dtype=torch.uint8, device=dev)
+                    if transposed else None))
+    fp8bw_quantize_weight_block_batch(ws, [o[0] for o in out], [o[1] for o in out],
+                                      [o[2] for o in out], stream, pow2=pow2)
+    return out

@@ -114,6 +114,28 @@ int fp8bw_quantize_weight_block(const uint16_t* w, int64_t n, int64_t k,
                                 uint8_t* q, float* s, uint8_t* q_t,
                                 void* stream);
 
+/* Several weights' 128x128 block quantisations in one launch (the weights of
+ * a layer, quantised once per step): each job is exactly what
+ * fp8bw_quantize_weight_block(w, n, k, q, s, q_t) computes; the tensors'
+ * tiles are walked by one persistent grid, so small weights share one
+ * launch's ramp and tail.
+ *   jobs  : HOST array of `count` job descriptions (read during the call
+ *           only); each job's pointers are device pointers as above.
+ *   count : 0..8 (0 is a no-op; more is FP8BW_ERR_SHAPE).
+ * Errors: a job's own checks as fp8bw_quantize_weight_block; besides, no
+ * output of any job may overlap any job's input or any other output
+ * (FP8BW_ERR_ALIAS). Nothing is launched when a check fails. */
+typedef struct fp8bw_weight_block_job {
+    const uint16_t* w;   /* bf16 [n, k]                                    */
+    int64_t n, k;
+    uint8_t* q;          /* E4M3 codes [n, k]                              */
+    float* s;            /* fp32 scales [ceil(n/128)][ceil(k/128)]         */
+    uint8_t* q_t;        /* E4M3 codes [k, n] (transposed) or NULL         */
+} fp8bw_weight_block_job;
+
+int fp8bw_quantize_weight_block_batch(const fp8bw_weight_block_job* jobs,
+                                      int count, void* stream);
+
 /* fprop: Y[m, n] = bf16( sum_c sX[c][m] * sW[n/128][c] *
  *                        sum_{kk in chunk c} qX[m, kk] * qW[n, kk] )
  *   qx, sx : row-wise quantised X: [m, k], [ceil(k/128)][m]
@@ -246,6 +268,8 @@ int fp8bw_quantize_colwise_pow2(const uint16_t* x, int64_t rows, int64_t cols,
 int fp8bw_quantize_weight_block_pow2(const uint16_t* w, int64_t n, int64_t k,
                                      uint8_t* q, float* s, uint8_t* q_t,
                                      void* stream);
+int fp8bw_quantize_weight_block_batch_pow2(const fp8bw_weight_block_job* jobs,
+                                           int count, void* stream);
 int fp8bw_gemm_fprop_pow2(const uint8_t* qx, const float* sx,
                           const uint8_t* qw, const float* sw, int64_t m,
                           int64_t n, int64_t k, uint16_t* y, void* stream);

@@ -37,14 +37,14 @@ def lib():
 
 def test_every_declared_symbol_is_exported(lib):
     names = declared_functions()
-    assert len(names) == 22
+    assert len(names) == 24
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(_native.SIGNATURES)
 
 
 def test_status_strings_and_version(lib):
-    assert lib.fp8bw_version() == 106
+    assert lib.fp8bw_version() == 107
     for st in (OK, E_NULL, E_SHAPE, E_ALIGN, E_DEVICE, E_LAUNCH, E_TIMEOUT,
                E_CUDA, E_ALIAS, E_SCALE):
         s = lib.fp8bw_status_string(st).decode()
@@ -156,10 +156,37 @@ def test_aliased_outputs_rejected(lib):
                                     None) == E_ALIAS
 
 
+def _jobs(*specs):
+    arr = (_native.WeightBlockJob * max(1, len(specs)))()
+    for i, sp in enumerate(specs):
+        arr[i] = _native.WeightBlockJob(*sp)
+    return ctypes.cast(arr, ctypes.c_void_p), arr
+
+
+def test_weight_block_batch_checks(lib):
+    ok1 = (A, 256, 128, B, C, D)                  # w, n, k, q, s, q_t
+    ok2 = (A + 0x100000, 128, 256, B + 0x100000, C + 0x100000, None)
+    p, keep = _jobs(ok1, ok2)
+    assert lib.fp8bw_quantize_weight_block_batch(p, 9, None) == E_SHAPE
+    assert lib.fp8bw_quantize_weight_block_batch(p, -1, None) == E_SHAPE
+    assert lib.fp8bw_quantize_weight_block_batch(None, 2, None) == E_NULL
+    p, keep = _jobs(ok1, (A + 0x100000, 100, 256, B + 0x100000, C + 0x100000, None))
+    assert lib.fp8bw_quantize_weight_block_batch(p, 2, None) == E_SHAPE
+    p, keep = _jobs(ok1, (A + 0x100000, 128, 256, B + 0x100008, C + 0x100000, None))
+    assert lib.fp8bw_quantize_weight_block_batch_pow2(p, 2, None) == E_ALIGN
+    # job 2's codes on top of job 1's input, and two jobs sharing a scale buffer
+    p, keep = _jobs(ok1, (A + 0x100000, 128, 256, A + 256, C + 0x100000, None))
+    assert lib.fp8bw_quantize_weight_block_batch(p, 2, None) == E_ALIAS
+    p, keep = _jobs(ok1, (A + 0x100000, 128, 256, B + 0x100000, C, None))
+    assert lib.fp8bw_quantize_weight_block_batch(p, 2, None) == E_ALIAS
+
+
 @pytest.mark.skipif(
     __import__("torch").cuda.is_available(),
     reason="checks the no-device path; on a GPU host the call would launch")
 def test_valid_call_without_device_reports_device_error(lib):
+    p, keep = _jobs((A, 256, 128, B, C, D))
+    assert lib.fp8bw_quantize_weight_block_batch(p, 1, None) == E_DEVICE
     assert lib.fp8bw_quantize_rowwise(A, 128, 128, B, C, None) == E_DEVICE
     assert lib.fp8bw_gemm_fprop(A, B, C, D, 128, 128, 128, E,
                                 None) == E_DEVICE

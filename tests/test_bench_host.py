@@ -70,7 +70,7 @@ class _FakeLibrary:
         if not name.startswith("fp8bw_"):
             raise AttributeError(name)
 
-        def call(*args):
+        def call(*args, **kwargs):
             self.calls[name] = self.calls.get(name, 0) + 1
         return call
 
@@ -79,13 +79,15 @@ class _FakeLinear:
     def __init__(self, kind, k, n):
         import torch
         self.kind, self.k, self.n = kind, k, n
-        for attr in ("qx", "sx", "qw", "sw", "qw_t", "qdy", "sdy", "qdy_t",
+        for attr in ("w", "qx", "sx", "qw", "sw", "qw_t", "qdy", "sdy", "qdy_t",
                      "sdy_t", "qx_t", "sx_t", "y", "dx"):
             setattr(self, attr, torch.zeros(1))
 
+    def weight_bytes(self):
+        return 1e6
+
     def ops(self, o, stream, pow2=False):
-        return [("quant_weight_block", 1e6, lambda: None),
-                ("quant_rowcol", 1e6, lambda: None),
+        return [("quant_rowcol", 1e6, lambda: None),
                 ("gemm_block_scaled", 1e9, lambda: None),
                 ("gemm_vector_scaled", 1e9, lambda: None)]
 

@@ -163,3 +163,22 @@ def test_newer_outputs_write_exactly_their_outputs(m, n, k):
     assert all(_eq(a, b) for a, b in zip((y, qy, sy, qy_t, sy_t), r))
     r = ops.gemm_dgrad_quant_rowcol(qdy, sdy, qw_t, sw)
     assert all(_eq(a, b) for a, b in zip((dx, qdx, sdx, qdx_t, sdx_t), r))
+
+
+@pytest.mark.parametrize("pow2", [False, True])
+def test_weight_block_batch_writes_exactly_its_outputs(pow2):
+    import torch
+    ops = _ops()
+    shapes = [(272, 400), (16, 16), (1040, 144), (384, 1296)]
+    ws = [bf16_np_to_torch(S.bf16_normal(sh, 0, 995 + i, **S.W_DIST))
+          for i, sh in enumerate(shapes)]
+    cd = lambda a: (a + 127) // 128  # noqa: E731
+    g = Guarded()
+    qs = [g.make(sh, torch.uint8) for sh in shapes]
+    ss = [g.make((cd(sh[0]), cd(sh[1])), torch.float32) for sh in shapes]
+    qts = [g.make((sh[1], sh[0]), torch.uint8) for sh in shapes]
+    ops.fp8bw_quantize_weight_block_batch(ws, qs, ss, qts, pow2=pow2)
+    g.check("batched weight quantisation")
+    for w, q, s, q_t in zip(ws, qs, ss, qts):
+        rq, rs, rq_t = ops.quantize_weight_block(w, pow2=pow2)
+        assert _eq(q, rq) and _eq(s, rs) and _eq(q_t, rq_t)

@@ -8,7 +8,7 @@ import pytest
 
 import oracle
 import synthetic as S
-from helpers import bf16_np_to_torch, hand_groups, scale_bits
+from helpers import bf16_np_to_torch, hand_groups, scale_bits, torch_bf16_to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -176,3 +176,35 @@ def test_full_size_activation_quantisers(name):
         _check_colwise(x, True)
         _check_weight(S.draw_w(lin))
     _ops().fp8bw_check_device_error()
+
+
+@pytest.mark.parametrize("pow2", [False, True])
+def test_weight_block_batch_equals_one_by_one(pow2):
+    """Several weights in one launch (ragged shapes, an empty one, with and
+    without transposed codes): each job's codes and scales equal, bit for bit,
+    the single-weight quantiser's and the oracle's."""
+    import torch
+    ops = _ops()
+    shapes = [(12288, 2048), (272, 400), (0, 256), (2048, 6144), (16, 16), (1040, 48)]
+    ws = [bf16_np_to_torch(S.bf16_normal(sh, 0, 560 + i, 0.02)) if sh[0] else
+          torch.empty(sh, dtype=torch.bfloat16, device="cuda")
+          for i, sh in enumerate(shapes)]
+    outs = ops.quantize_weight_block_batch(ws, pow2=pow2)
+    qts = [o[2] for o in outs]
+    qts[3] = None                        # one job without transposed codes
+    qs = [o[0] for o in outs]
+    ss = [o[1] for o in outs]
+    ops.fp8bw_quantize_weight_block_batch(ws, qs, ss, qts, pow2=pow2)
+    ops.fp8bw_check_device_error()
+    for i, (w, q, s) in enumerate(zip(ws, qs, ss)):
+        if w.numel() == 0:
+            continue
+        rq, rs, rq_t = ops.quantize_weight_block(w, pow2=pow2)
+        assert torch.equal(q, rq), i
+        assert torch.equal(s.view(torch.int32), rs.view(torch.int32)), i
+        if qts[i] is not None:
+            assert torch.equal(qts[i], rq_t), i
+        if w.shape[0] * w.shape[1] <= 1 << 22:
+            oq, os_, _ = oracle.quantize_weight_block(torch_bf16_to_np(w), pow2=pow2)
+            assert np.array_equal(q.cpu().numpy(), oq), i
+            assert np.array_equal(scale_bits(s.cpu().numpy()), scale_bits(os_)), i
