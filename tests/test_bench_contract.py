@@ -51,4 +51,4 @@ def test_gpu_arm_line_one_layer():
     assert e["value"] > 0 and e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] > 0
     assert d["clocks"] is None or d["clocks"]["sm_mhz"] > 0
     assert set(d["next_rows"]) == {"wgrad_f32_accumulate", "gemm_fused_rowwise_quant",
-                                   "pow2_step"}
+                                   "gemm_fused_rowcol_quant", "pow2_step"}
