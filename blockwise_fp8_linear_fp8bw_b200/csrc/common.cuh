@@ -181,6 +181,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Both phases complete? The two probes are issued back to back, so their
+// latencies (a shared-memory round trip each, long when the tensor cores and
+// TMA keep shared memory busy) overlap instead of adding up.
+__device__ __forceinline__ bool mbar_try_wait2(uint32_t bar1, uint32_t parity1, uint32_t bar2,
+                                               uint32_t parity2) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p1, p2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p1, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p2, [%3], %4;\n\t"
+      "and.pred p1, p1, p2;\n\t"
+      "selp.u32 %0, 1, 0, p1;\n\t}"
+      : "=r"(ok)
+      : "r"(bar1), "r"(parity1), "r"(bar2), "r"(parity2)
+      : "memory");
+  return ok != 0;
+}
+
 // As mbar_try_wait, but a thread whose phase is not complete yet is suspended
 // (not spinning on issue slots) until it completes or `suspend_ns` elapse.
 __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,

@@ -69,7 +69,6 @@ namespace gemm {
 constexpr int BM = 128;           // tile rows (UMMA M)
 constexpr int BK = 128;           // contraction chunk = scale group length
 constexpr int kStages = 4;        // A/B smem ring depth
-constexpr int kScaleStages = 8;   // scale ring depth
 constexpr int kThreads = 384;
 constexpr int kFirstEpiWarp = 4;
 constexpr int kNumEpiWarps = 8;
@@ -117,6 +116,10 @@ struct PairLayout {
   static constexpr int kBBytes = (BN / 2) * BK;  // this CTA's BN/2 B rows
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kRingBytes = kStages * kStageBytes;
+  // scale ring depth: the scales are small, but their loads wait behind the
+  // operand traffic, so the ring runs far ahead (fewer slots in vector mode,
+  // whose slots also hold BN column scales)
+  static constexpr int kScaleStages = VEC_B ? 8 : 16;
   static constexpr int kSaBytes = BM * 4;
   static constexpr int kSbBytes = VEC_B ? BN * 4 : 16;
   static constexpr int kScaleSlot = kSaBytes + kSbBytes;
@@ -144,6 +147,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                const Args g) {
   using L = PairLayout<BN_, VEC_B>;
   constexpr int BN = L::BN;
+  constexpr int kScaleStages = L::kScaleStages;
   constexpr int kPairStages = L::kStages;
   constexpr int kBufs = L::kTmemBufs;
   static_assert(!B_MN || BN == 256, "MN-major B uses full 128-element swizzle atoms");
@@ -275,8 +279,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint32_t u = it / kPairStages;
           const int tb = tc % kBufs;
           const uint32_t tu = tc / kBufs;
-          if (!mbar_wait(full_bar(s), u & 1u, abort_flag, kErrTimeoutMma) ||
-              !mbar_wait(tempty_bar(tb), (tu & 1u) ^ 1u, abort_flag, kErrTimeoutMma)) {
+          if (!mbar_try_wait2(full_bar(s), u & 1u, tempty_bar(tb), (tu & 1u) ^ 1u) &&
+              (!mbar_wait(full_bar(s), u & 1u, abort_flag, kErrTimeoutMma) ||
+               !mbar_wait(tempty_bar(tb), (tu & 1u) ^ 1u, abort_flag, kErrTimeoutMma))) {
             ok = false;
             break;
           }
@@ -307,6 +312,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ scale producer
+    // Block mode: the weight-block scales of this CTA's sequence of chunks
+    // (tile after tile), 32 chunks per window; lane l holds chunk 32w + l of
+    // window w. The next window is loaded as the current one starts, so the
+    // global loads have 32 chunks to land.
+    auto load_window = [&](int w, float& p0, float& p1) {
+      p0 = 0.0f;
+      p1 = 0.0f;
+      const int64_t fi = static_cast<int64_t>(w) * 32 + lane;
+      const int64_t k = fi / C;
+      const int cc = static_cast<int>(fi - k * C);
+      const int64_t t = cluster_id + k * num_clusters;
+      if (t < num_tiles) {
+        const int jb0 = static_cast<int>(t % g.tiles_n) * (BN / 128);
+        p0 = __ldg(g.sb + jb0 * g.sbj + static_cast<int64_t>(cc) * g.sbc);
+        if (BN > 128 && jb0 + 1 < g.nblk)
+          p1 = __ldg(g.sb + (jb0 + 1) * g.sbj + static_cast<int64_t>(cc) * g.sbc);
+      }
+    };
+    float cur0 = 0.0f, cur1 = 0.0f, nxt0 = 0.0f, nxt1 = 0.0f;
+    if constexpr (!VEC_B) {
+      load_window(0, cur0, cur1);
+      load_window(1, nxt0, nxt1);
+    }
     uint32_t sit = 0;
     bool ok = true;
     for (int tile = cluster_id; ok && tile < num_tiles; tile += num_clusters) {
@@ -315,23 +343,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int rows_here = max(0, min(BM, g.mo - m0));
       const uint32_t a_bytes = static_cast<uint32_t>(rows_here) * 4u;
       const uint32_t b_bytes = VEC_B ? static_cast<uint32_t>(min(BN, g.no - n0)) * 4u : 0u;
-      const int jb0 = n0 / 128;
-      float pre0 = 0.0f, pre1 = 0.0f;
       for (int c = 0; c < C; ++c, ++sit) {
         if constexpr (!VEC_B) {
-          if ((c & 31) == 0) {
-            const int cc = c + lane;
-            pre0 = 0.0f;
-            pre1 = 0.0f;
-            if (cc < C) {
-              pre0 = g.sb[jb0 * g.sbj + static_cast<int64_t>(cc) * g.sbc];
-              if (BN > 128 && jb0 + 1 < g.nblk)
-                pre1 = g.sb[(jb0 + 1) * g.sbj + static_cast<int64_t>(cc) * g.sbc];
-            }
+          if ((sit & 31u) == 0 && sit > 0) {
+            cur0 = nxt0;
+            cur1 = nxt1;
+            load_window(static_cast<int>(sit >> 5) + 1, nxt0, nxt1);
           }
         }
-        const float v0 = __shfl_sync(0xFFFFFFFFu, pre0, c & 31);
-        const float v1 = __shfl_sync(0xFFFFFFFFu, pre1, c & 31);
+        const float v0 = __shfl_sync(0xFFFFFFFFu, cur0, sit & 31u);
+        const float v1 = __shfl_sync(0xFFFFFFFFu, cur1, sit & 31u);
         uint32_t good = 1u;
         if (lane == 0) {
           const int ss = sit % kScaleStages;
@@ -393,19 +414,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t tu = tc >> 1;
         const int ss = sit % kScaleStages;
         const uint32_t su = sit / kScaleStages;
-        if (!mbar_wait(tfull_bar(tb), tu & 1u, abort_flag, kErrTimeoutEpi) ||
-            !mbar_wait(sfull_bar(ss), su & 1u, abort_flag, kErrTimeoutEpi)) {
+        // fast path: both phases already complete (one overlapped probe)
+        if (!mbar_try_wait2(tfull_bar(tb), tu & 1u, sfull_bar(ss), su & 1u) &&
+            (!mbar_wait(tfull_bar(tb), tu & 1u, abort_flag, kErrTimeoutEpi) ||
+             !mbar_wait(sfull_bar(ss), su & 1u, abort_flag, kErrTimeoutEpi))) {
           ok = false;
           break;
         }
         tc_fence_after();
         const float* slot = reinterpret_cast<const float*>(smem + L::kScaleOff + ss * L::kScaleSlot);
         const float* sbv = slot + BM;                 // B scales of this chunk
-        uint64_t blk2 = 0ull;
-        if constexpr (!VEC_B) {
-          const uint32_t b = __float_as_uint(slot[row] * sbv[BN > 128 ? h : 0]);
-          blk2 = pack2(b, b);
-        }
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                static_cast<uint32_t>(tb * BN + h * kHalf);
         if constexpr (VEC_B) {
@@ -416,8 +434,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           // shared-memory reads of those dominated).
           const int g4 = lane >> 2, c4 = lane & 3;
           float sa4[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) sa4[i] = slot[q * 32 + g4 + 8 * i];
           float* af = reinterpret_cast<float*>(acc2);   // [i][p][2]
 #pragma unroll
           for (int part = 0; part < 2; ++part) {
@@ -425,6 +441,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tmem_ld16x256_x8(taddr + part * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
             tmem_ld16x256_x8(taddr + (16u << 16) + part * 64,
                              *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+            // scales read while the TMEM loads are in flight
+            if (part == 0) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) sa4[i] = slot[q * 32 + g4 + 8 * i];
+            }
+            float2 bcol[4];
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr)
+              bcol[rr] = *reinterpret_cast<const float2*>(sbv + h * kHalf + 8 * (part * 8 + rr) + 2 * c4);
             tmem_wait_ld();
             tmem_regs_ready(r);
             if (part == 1) {
@@ -435,7 +460,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int rr = 0; rr < 8; ++rr) {
               const int p = part * 8 + rr;
-              const float2 b = *reinterpret_cast<const float2*>(sbv + h * kHalf + 8 * p + 2 * c4);
+              const float2 b = rr < 4 ? bcol[rr]
+                                      : *reinterpret_cast<const float2*>(sbv + h * kHalf + 8 * p + 2 * c4);
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
                 // rows g4, g4+8 from the first load, g4+16, g4+24 from the second
@@ -448,11 +474,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
           }
         } else {
+          uint64_t blk2 = 0ull;
 #pragma unroll
           for (int part = 0; part < kHalf / 64; ++part) {
             uint32_t r[64];
             tmem_ld32(taddr + part * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
             tmem_ld32(taddr + part * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+            if (part == 0) {
+              // the scales are read while the first TMEM load is in flight
+              const uint32_t b = __float_as_uint(slot[row] * sbv[BN > 128 ? h : 0]);
+              blk2 = pack2(b, b);
+            }
             tmem_wait_ld();
             tmem_regs_ready(r);
             if (part == kHalf / 64 - 1) {
