@@ -66,6 +66,13 @@
 namespace fp8bw {
 namespace gemm {
 
+#ifndef FP8BW_GEMM_STAGES
+#define FP8BW_GEMM_STAGES 4       // operand ring depth (256-wide tiles)
+#endif
+#ifndef FP8BW_OUT_BOXES
+#define FP8BW_OUT_BOXES 4         // output staging boxes per promotion warp
+#endif
+
 constexpr int BM = 128;           // tile rows (UMMA M)
 constexpr int BK = 128;           // contraction chunk = scale group length
 constexpr int kStages = 4;        // A/B smem ring depth
@@ -110,7 +117,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 template <int BN_, bool VEC_B>
 struct PairLayout {
   static constexpr int BN = BN_;                 // pair tile columns (128 or 256)
-  static constexpr int kStages = BN == 256 ? 6 : 8;
+  static constexpr int kStages = BN == 256 ? FP8BW_GEMM_STAGES : 8;
   static constexpr int kTmemBufs = 512 / BN;     // fp32 partial buffers in TMEM
   static constexpr int kABytes = BM * BK;        // this CTA's 128 A rows
   static constexpr int kBBytes = (BN / 2) * BK;  // this CTA's BN/2 B rows
@@ -128,10 +135,11 @@ struct PairLayout {
   // + 2 x 2 column-max barriers (column half, double buffer) for kOutBf16QQ
   static constexpr int kNumBars = 2 * kStages + 2 * kScaleStages + 2 * kTmemBufs + 1 + 4;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kOutWarpBytes = 32 * 32 * 2;
+  static constexpr int kOutWarpBytes = 32 * 32 * 2;        // one staging box
+  static constexpr int kOutBoxes = FP8BW_OUT_BOXES;         // staging boxes per warp
   static constexpr int kOutOff = ((kMiscOff + 16 + 1023) / 1024) * 1024;
   // kOutBf16QQ: per column half and buffer, 4 warps x 32 column maxima
-  static constexpr int kColMaxOff = kOutOff + kNumEpiWarps * kOutWarpBytes;
+  static constexpr int kColMaxOff = kOutOff + kNumEpiWarps * kOutBoxes * kOutWarpBytes;
   static constexpr int kColMaxBytes = 2 * 2 * 4 * 32 * 4;
   static constexpr int kBytes = kColMaxOff + kColMaxBytes;
   static constexpr int kAlloc = kBytes + 1024;
@@ -398,7 +406,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int ew = warp - kFirstEpiWarp;
     const int h = ew >> 2;                           // column half of the tile
     const int row = q * 32 + lane;                   // this CTA's tile row = TMEM lane
-    const uint32_t stage_out = sbase + L::kOutOff + ew * L::kOutWarpBytes;
+    const uint32_t stage_out = sbase + L::kOutOff + ew * L::kOutBoxes * L::kOutWarpBytes;
+    uint32_t out_seq = 0;         // boxes this warp has staged
     const uint32_t tempty_leader0 = mapa_shared(tempty_bar(0), 0);
     uint32_t tc = 0, sit = 0;
     uint32_t box_seq = 0;         // kOutBf16QQ: boxes this warp has quantised
@@ -534,8 +543,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // rows are all past the end still takes part (it stores nothing).
         if (x0 + gi * kBoxCols >= g.no) continue;
         if (OUT != kOutBf16QQ && y0 >= g.mo) continue;
+        // the box that used this staging buffer kOutBoxes stores ago must
+        // have been read by its TMA store
+        const uint32_t stage_box = stage_out + (out_seq % L::kOutBoxes) * L::kOutWarpBytes;
+        ++out_seq;
         if (store_pending) {
-          if (lane == 0) bulk_wait_group_read<0>();
+          if (lane == 0) bulk_wait_group_read<L::kOutBoxes - 1>();
           __syncwarp();
         }
         if constexpr (VEC_B) {
@@ -545,7 +558,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int R = g4 + 8 * i;
-            const uint32_t rowp = stage_out + R * 64;
+            const uint32_t rowp = stage_box + R * 64;
             const uint32_t sw = (R >> 1) & 3;
             if constexpr (OUT == kOutBf16) {
 #pragma unroll
@@ -593,7 +606,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               w2 = __float_as_uint(v[2]);
               w3 = __float_as_uint(v[3]);
             }
-            const uint32_t dst = stage_out + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4);
+            const uint32_t dst = stage_box + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4);
             asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(w0),
                          "r"(w1), "r"(w2), "r"(w3)
                          : "memory");
@@ -626,7 +639,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int e = 0; e < 2; ++e) {
                 const int rr = 2 * i + e;
-                const uint32_t addr = stage_out + rr * 64 +
+                const uint32_t addr = stage_box + rr * 64 +
                                       (((lane >> 3) ^ ((rr >> 1) & 3)) << 4) + (lane & 7) * 2;
                 uint16_t hv;
                 asm volatile("ld.shared.u16 %0, [%1];" : "=h"(hv) : "r"(addr) : "memory");
@@ -674,9 +687,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) {
           if constexpr (OUT == kOutF32Add)
-            tma_reduce_add_2d(&tm_out, stage_out, x0 + gi * kBoxCols, y0);
+            tma_reduce_add_2d(&tm_out, stage_box, x0 + gi * kBoxCols, y0);
           else
-            tma_store_2d(&tm_out, stage_out, x0 + gi * kBoxCols, y0);
+            tma_store_2d(&tm_out, stage_box, x0 + gi * kBoxCols, y0);
           bulk_commit_group();
         }
         store_pending = true;
