@@ -338,8 +338,10 @@ class LinearBuffers:
 
     def ops(self, o, stream, pow2=False):
         """[(kernel kind, algorithmic units, callable)] of this linear after
-        its weight is quantised (layer_ops quantises a layer's weights in one
-        launch); pow2 selects the power-of-two-scale quantisers and GEMMs."""
+        its weight is quantised and before its weight gradient (layer_ops
+        quantises a layer's weights in one launch and computes its weight
+        gradients in another); pow2 selects the power-of-two-scale quantisers
+        and GEMMs."""
         m, k, n = TOKENS, self.k, self.n
         cd = lambda a: (a + 127) // 128  # noqa: E731
         xq_bytes = m * k * 2 + 2 * m * k + 4 * (m * cd(k) + cd(m) * k)
@@ -361,16 +363,19 @@ class LinearBuffers:
             ("gemm_block_scaled", f,
              lambda: o.fp8bw_gemm_dgrad(self.qdy, self.sdy, self.qw_t, 1,
                                         self.sw, self.dx, stream, pow2=p2)),
-            ("gemm_vector_scaled", f,
-             lambda: o.fp8bw_gemm_wgrad(self.qdy_t, self.sdy_t, self.qx_t,
-                                        self.sx_t, self.dw, stream, pow2=p2)),
         ]
+
+    def wgrad_job(self):
+        """(qdy_t, sdy_t, qx_t, sx_t, dw) of this linear's weight gradient."""
+        return (self.qdy_t, self.sdy_t, self.qx_t, self.sx_t, self.dw)
 
 
 def layer_ops(bufs, o, stream, pow2=False):
     """The ops of one layer: its weights' 128x128 block quantisation in one
     launch (all weights are quantised once per step, before they are used),
-    then each linear's quantisers and GEMMs."""
+    then each linear's quantisers, fprop and dgrad, then the weight gradients
+    of all its linears in one launch (they contract over the same tokens; a
+    backward pass can defer them until the layer's dY are all known)."""
     ws = [b.w for b in bufs]
     qs, ss, qts = [b.qw for b in bufs], [b.sw for b in bufs], [b.qw_t for b in bufs]
     out = [("quant_weight_block", sum(b.weight_bytes() for b in bufs),
@@ -378,6 +383,9 @@ def layer_ops(bufs, o, stream, pow2=False):
                                                         pow2=pow2))]
     for b in bufs:
         out.extend(b.ops(o, stream, pow2=pow2))
+    out.append(("gemm_vector_scaled", sum(2 * TOKENS * b.n * b.k for b in bufs),
+                lambda: o.fp8bw_gemm_wgrad_batch([b.wgrad_job() for b in bufs],
+                                                 stream, pow2=pow2)))
     return out
 
 
@@ -393,16 +401,16 @@ def linear_names(kinds):
 def time_next_rows(o, bufs, stream, warmup, rounds):
     """Rows beyond the step, timed after it on the same buffers (not part of
     `value`): wgrad with an fp32 dW added into an fp32 main-grad buffer, the
-    four linears of a layer in turn (their operands together exceed L2)."""
+    four linears of a layer in one launch (their operands together exceed
+    L2)."""
     import torch
     dev = bufs[0].qx_t.device
     names = linear_names([b.kind for b in bufs])
     grads = [torch.zeros((b.n, b.k), dtype=torch.float32, device=dev)
              for b in bufs]
-    calls = [(2 * TOKENS * b.n * b.k,
-              (lambda b=b, g=g: o.fp8bw_gemm_wgrad_f32(
-                  b.qdy_t, b.sdy_t, b.qx_t, b.sx_t, g, True, stream)))
-             for b, g in zip(bufs, grads)]
+    jobs = [b.wgrad_job()[:4] + (g,) for b, g in zip(bufs, grads)]
+    calls = [(sum(2 * TOKENS * b.n * b.k for b in bufs),
+              lambda: o.fp8bw_gemm_wgrad_f32_batch(jobs, True, stream))]
     with torch.cuda.stream(stream):
         for _ in range(warmup):
             for _, fn in calls:
@@ -424,8 +432,8 @@ def time_next_rows(o, bufs, stream, warmup, rounds):
     out = {"wgrad_f32_accumulate": {
         "achieved": flop / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
         "launches": rounds * len(calls), "avg_launch_ms": ms / (rounds * len(calls)),
-        "what": "dW (fp32) += dY^T X for the %s linears at M=%d, in turn; "
-                "timed after the step" % (names, TOKENS)}}
+        "what": "dW (fp32) += dY^T X for the %s linears at M=%d, one "
+                "launch for all; timed after the step" % (names, TOKENS)}}
 
     # fprop and dgrad that also quantise their own bf16 output row-wise,
     # against the same GEMMs followed by the row-wise quantiser.

@@ -18,6 +18,12 @@ class WeightBlockJob(ctypes.Structure):
                 ("q_t", _P)]
 
 
+class WgradJob(ctypes.Structure):
+    """fp8bw_wgrad_job of include/fp8bw.h."""
+    _fields_ = [("qdy_t", _P), ("sdy_t", _P), ("qx_t", _P), ("sx_t", _P),
+                ("m", _I64), ("n", _I64), ("k", _I64), ("dw", _P)]
+
+
 # name -> (argtypes, restype), in the order of include/fp8bw.h
 SIGNATURES = {
     "fp8bw_quantize_rowwise": ([_P, _I64, _I64, _P, _P, _P], _INT),
@@ -30,6 +36,8 @@ SIGNATURES = {
     "fp8bw_gemm_wgrad": ([_P, _P, _P, _P, _I64, _I64, _I64, _P, _P], _INT),
     "fp8bw_gemm_wgrad_f32": ([_P, _P, _P, _P, _I64, _I64, _I64, _P, _INT,
                               _P], _INT),
+    "fp8bw_gemm_wgrad_batch": ([_P, _INT, _P], _INT),
+    "fp8bw_gemm_wgrad_f32_batch": ([_P, _INT, _INT, _P], _INT),
     "fp8bw_gemm_fprop_quant": ([_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P,
                                 _P], _INT),
     "fp8bw_gemm_dgrad_quant": ([_P, _P, _P, _INT, _P, _I64, _I64, _I64, _P, _P,
@@ -48,6 +56,8 @@ SIGNATURES = {
     "fp8bw_gemm_wgrad_pow2": ([_P, _P, _P, _P, _I64, _I64, _I64, _P, _P], _INT),
     "fp8bw_gemm_wgrad_f32_pow2": ([_P, _P, _P, _P, _I64, _I64, _I64, _P, _INT,
                                    _P], _INT),
+    "fp8bw_gemm_wgrad_batch_pow2": ([_P, _INT, _P], _INT),
+    "fp8bw_gemm_wgrad_f32_batch_pow2": ([_P, _INT, _INT, _P], _INT),
     "fp8bw_selftest_wait_timeout": ([_I64, _P], _INT),
     "fp8bw_check_device_error": ([_P], _INT),
     "fp8bw_status_string": ([_INT], ctypes.c_char_p),

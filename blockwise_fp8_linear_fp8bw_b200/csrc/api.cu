@@ -202,11 +202,14 @@ struct GemmProblem {
   float* st_out;     // kOutBf16QQ: their scales [ceil(mo/128)][no]
 };
 
-// CTA-pair kernel: 256 x 256 output tiles on clusters of two CTAs.
-template <int BN, bool VEC_B, bool B_MN, int OUT = kOutBf16>
-int launch_gemm_pair(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t stream) {
+// CTA-pair kernel: 256 x 256 output tiles on clusters of two CTAs, over
+// `count` (1..NJ) problems of the same form and contraction length.
+template <int BN, bool VEC_B, bool B_MN, int OUT = kOutBf16, int NJ = 1>
+int launch_gemm_pair(const GemmProblem* ps, int count, const DeviceInfo& dev,
+                     cudaStream_t stream) {
   using L = gemm::PairLayout<BN, VEC_B>;
-  auto kernel = gemm::blockwise_gemm_pair_kernel<BN, VEC_B, B_MN, OUT>;
+  auto kernel = gemm::blockwise_gemm_pair_kernel<BN, VEC_B, B_MN, OUT, NJ>;
+  if (count < 1 || count > NJ) return FP8BW_ERR_LAUNCH;
   static DevicePrep prep;
   int max_clusters = 0;
   const int prep_status = prepare_for_device(prep, dev.ordinal, &max_clusters, [&](int* mc) {
@@ -225,44 +228,57 @@ int launch_gemm_pair(const GemmProblem& p, const DeviceInfo& dev, cudaStream_t s
   });
   if (prep_status != FP8BW_OK) return prep_status;
 
-  CUtensorMap tm_a, tm_b, tm_out;
-  int st = encode_u8_2d(&tm_a, p.a, static_cast<uint64_t>(p.kc), static_cast<uint64_t>(p.mo),
-                        gemm::BM);
-  if (st != FP8BW_OK) return st;
-  if (B_MN)
-    st = encode_u8_2d(&tm_b, p.b, static_cast<uint64_t>(p.no), static_cast<uint64_t>(p.kc), 128);
-  else
-    st = encode_u8_2d(&tm_b, p.b, static_cast<uint64_t>(p.kc), static_cast<uint64_t>(p.no),
-                      BN / 2);
-  if (st != FP8BW_OK) return st;
-  if (out_is_bf16(OUT))
-    st = encode_bf16_out(&tm_out, p.out, static_cast<uint64_t>(p.no),
-                         static_cast<uint64_t>(p.mo));
-  else
-    st = encode_f32_out(&tm_out, p.out, static_cast<uint64_t>(p.no), static_cast<uint64_t>(p.mo));
-  if (st != FP8BW_OK) return st;
+  gemm::PairMaps<NJ> maps;
+  gemm::PairArgs<NJ> pa;
+  std::memset(&maps, 0, sizeof maps);
+  std::memset(&pa, 0, sizeof pa);
+  int64_t tiles = 0;
+  for (int i = 0; i < count; ++i) {
+    const GemmProblem& p = ps[i];
+    int st = encode_u8_2d(&maps.a[i], p.a, static_cast<uint64_t>(p.kc),
+                          static_cast<uint64_t>(p.mo), gemm::BM);
+    if (st != FP8BW_OK) return st;
+    if (B_MN)
+      st = encode_u8_2d(&maps.b[i], p.b, static_cast<uint64_t>(p.no), static_cast<uint64_t>(p.kc),
+                        128);
+    else
+      st = encode_u8_2d(&maps.b[i], p.b, static_cast<uint64_t>(p.kc), static_cast<uint64_t>(p.no),
+                        BN / 2);
+    if (st != FP8BW_OK) return st;
+    if (out_is_bf16(OUT))
+      st = encode_bf16_out(&maps.out[i], p.out, static_cast<uint64_t>(p.no),
+                           static_cast<uint64_t>(p.mo));
+    else
+      st = encode_f32_out(&maps.out[i], p.out, static_cast<uint64_t>(p.no),
+                          static_cast<uint64_t>(p.mo));
+    if (st != FP8BW_OK) return st;
 
-  gemm::Args g;
-  g.mo = static_cast<int>(p.mo);
-  g.no = static_cast<int>(p.no);
-  g.kc = static_cast<int>(p.kc);
-  g.tiles_m = static_cast<int>(cdiv(p.mo, 2 * gemm::BM));
-  g.tiles_n = static_cast<int>(cdiv(p.no, L::BN));
-  g.chunks = static_cast<int>(cdiv(p.kc, gemm::BK));
-  g.sa = p.sa;
-  g.sb = p.sb;
-  g.sbj = p.sbj;
-  g.sbc = p.sbc;
-  g.nblk = static_cast<int>(cdiv(p.no, 128));
-  g.out = p.out;
-  g.q_out = p.q_out;
-  g.s_out = p.s_out;
-  g.qt_out = p.qt_out;
-  g.st_out = p.st_out;
-  const int64_t tiles = static_cast<int64_t>(g.tiles_m) * g.tiles_n;
+    gemm::Args& g = pa.job[i];
+    g.mo = static_cast<int>(p.mo);
+    g.no = static_cast<int>(p.no);
+    g.kc = static_cast<int>(p.kc);
+    g.tiles_m = static_cast<int>(cdiv(p.mo, 2 * gemm::BM));
+    g.tiles_n = static_cast<int>(cdiv(p.no, L::BN));
+    g.chunks = static_cast<int>(cdiv(p.kc, gemm::BK));
+    g.sa = p.sa;
+    g.sb = p.sb;
+    g.sbj = p.sbj;
+    g.sbc = p.sbc;
+    g.nblk = static_cast<int>(cdiv(p.no, 128));
+    g.out = p.out;
+    g.q_out = p.q_out;
+    g.s_out = p.s_out;
+    g.qt_out = p.qt_out;
+    g.st_out = p.st_out;
+    if (g.chunks != pa.job[0].chunks) return FP8BW_ERR_SHAPE;
+    tiles += static_cast<int64_t>(g.tiles_m) * g.tiles_n;
+    if (tiles > (int64_t(1) << 30)) return FP8BW_ERR_SHAPE;
+    pa.tile_end[i] = static_cast<int>(tiles);
+  }
+  for (int i = count; i < NJ; ++i) pa.tile_end[i] = static_cast<int>(tiles);
   const int clusters = static_cast<int>(std::min<int64_t>(tiles, max_clusters));
-  if (launch_kernel(kernel, dim3(2 * clusters), dim3(gemm::kThreads), L::kAlloc, stream, tm_a,
-                    tm_b, tm_out, g) != cudaSuccess)
+  if (launch_kernel(kernel, dim3(2 * clusters), dim3(gemm::kThreads), L::kAlloc, stream, maps, pa) !=
+      cudaSuccess)
     return FP8BW_ERR_LAUNCH;
   return cudaGetLastError() == cudaSuccess ? FP8BW_OK : FP8BW_ERR_LAUNCH;
 }
@@ -367,21 +383,21 @@ int run_gemm(const GemmProblem& p, cudaStream_t stream) {
     return launch_gemm_pow2<false, false>(p, dev, stream);
   }
   if (p.vec_b && p.out_mode == kOutF32)
-    return launch_gemm_pair<GEMM_BN_VEC, true, false, kOutF32>(p, dev, stream);
+    return launch_gemm_pair<GEMM_BN_VEC, true, false, kOutF32>(&p, 1, dev, stream);
   if (p.vec_b && p.out_mode == kOutF32Add)
-    return launch_gemm_pair<GEMM_BN_VEC, true, false, kOutF32Add>(p, dev, stream);
+    return launch_gemm_pair<GEMM_BN_VEC, true, false, kOutF32Add>(&p, 1, dev, stream);
   if (p.out_mode == kOutBf16Q && !p.vec_b) {
-    if (p.b_mn) return launch_gemm_pair<256, false, true, kOutBf16Q>(p, dev, stream);
-    return launch_gemm_pair<256, false, false, kOutBf16Q>(p, dev, stream);
+    if (p.b_mn) return launch_gemm_pair<256, false, true, kOutBf16Q>(&p, 1, dev, stream);
+    return launch_gemm_pair<256, false, false, kOutBf16Q>(&p, 1, dev, stream);
   }
   if (p.out_mode == kOutBf16QQ && !p.vec_b) {
-    if (p.b_mn) return launch_gemm_pair<256, false, true, kOutBf16QQ>(p, dev, stream);
-    return launch_gemm_pair<256, false, false, kOutBf16QQ>(p, dev, stream);
+    if (p.b_mn) return launch_gemm_pair<256, false, true, kOutBf16QQ>(&p, 1, dev, stream);
+    return launch_gemm_pair<256, false, false, kOutBf16QQ>(&p, 1, dev, stream);
   }
   if (p.out_mode != kOutBf16) return FP8BW_ERR_LAUNCH;
-  if (p.vec_b) return launch_gemm_pair<GEMM_BN_VEC, true, false>(p, dev, stream);
-  if (p.b_mn) return launch_gemm_pair<256, false, true>(p, dev, stream);
-  return launch_gemm_pair<GEMM_BN_BLOCK, false, false>(p, dev, stream);
+  if (p.vec_b) return launch_gemm_pair<GEMM_BN_VEC, true, false>(&p, 1, dev, stream);
+  if (p.b_mn) return launch_gemm_pair<256, false, true>(&p, 1, dev, stream);
+  return launch_gemm_pair<GEMM_BN_BLOCK, false, false>(&p, 1, dev, stream);
 }
 
 }  // namespace
@@ -391,7 +407,7 @@ using namespace fp8bw;
 
 extern "C" {
 
-int fp8bw_version(void) { return 107; }
+int fp8bw_version(void) { return 108; }
 
 const char* fp8bw_status_string(int status) {
   switch (status) {
@@ -735,9 +751,11 @@ int fp8bw_gemm_dgrad_pow2(const uint8_t* qdy, const float* sdy, const uint8_t* q
 
 namespace {
 
-int wgrad_common(const uint8_t* qdy_t, const float* sdy_t, const uint8_t* qx_t,
-                 const float* sx_t, int64_t m, int64_t n, int64_t k, void* dw, int out_mode,
-                 bool pow2, void* stream) {
+// Checks of one wgrad problem (sizes, pointers, alignment, dW not overlapping
+// an input) and its description for the GEMM launchers.
+int wgrad_problem(const uint8_t* qdy_t, const float* sdy_t, const uint8_t* qx_t,
+                  const float* sx_t, int64_t m, int64_t n, int64_t k, void* dw, int out_mode,
+                  bool pow2, GemmProblem* out) {
   if (!dim_ok(m) || !dim_ok(n) || !dim_ok(k)) return FP8BW_ERR_SHAPE;
   if (missing(qdy_t, n * m) || missing(sdy_t, cdiv(m, 128) * n) || missing(qx_t, k * m) ||
       missing(sx_t, cdiv(m, 128) * k) || missing(dw, n * k))
@@ -765,7 +783,74 @@ int wgrad_common(const uint8_t* qdy_t, const float* sdy_t, const uint8_t* qx_t,
   p.out = dw;
   p.out_mode = out_mode;
   p.pow2 = pow2;
+  *out = p;
+  return FP8BW_OK;
+}
+
+int wgrad_common(const uint8_t* qdy_t, const float* sdy_t, const uint8_t* qx_t,
+                 const float* sx_t, int64_t m, int64_t n, int64_t k, void* dw, int out_mode,
+                 bool pow2, void* stream) {
+  GemmProblem p{};
+  const int st = wgrad_problem(qdy_t, sdy_t, qx_t, sx_t, m, n, k, dw, out_mode, pow2, &p);
+  if (st != FP8BW_OK) return st;
   return run_gemm(p, static_cast<cudaStream_t>(stream));
+}
+
+// Several wgrad problems with the same token count m in one launch of the
+// software-promotion kernel (their tiles share one wave schedule); the
+// power-of-two kernel takes them one launch each.
+int wgrad_batch(const fp8bw_wgrad_job* jobs, int count, int out_mode, bool pow2,
+                void* stream) {
+  if (count < 0 || count > gemm::kMaxGemmJobs) return FP8BW_ERR_SHAPE;
+  if (count > 0 && jobs == nullptr) return FP8BW_ERR_NULL;
+  GemmProblem ps[gemm::kMaxGemmJobs];
+  Range ins[4 * gemm::kMaxGemmJobs], outs[gemm::kMaxGemmJobs];
+  const int64_t esize = out_is_bf16(out_mode) ? 2 : 4;
+  for (int i = 0; i < count; ++i) {
+    const fp8bw_wgrad_job& j = jobs[i];
+    const int st = wgrad_problem(j.qdy_t, j.sdy_t, j.qx_t, j.sx_t, j.m, j.n, j.k, j.dw,
+                                 out_mode, pow2, &ps[i]);
+    if (st != FP8BW_OK) return st;
+    if (j.m != jobs[0].m) return FP8BW_ERR_SHAPE;
+    ins[4 * i] = range_of(j.qdy_t, j.n * j.m);
+    ins[4 * i + 1] = range_of(j.sdy_t, cdiv(j.m, 128) * j.n * 4);
+    ins[4 * i + 2] = range_of(j.qx_t, j.k * j.m);
+    ins[4 * i + 3] = range_of(j.sx_t, cdiv(j.m, 128) * j.k * 4);
+    outs[i] = range_of(j.dw, j.n * j.k * esize);
+  }
+  // no dW may overlap any job's input or another dW
+  for (int o = 0; o < count; ++o) {
+    for (int i = 0; i < 4 * count; ++i)
+      if (overlap(outs[o], ins[i])) return FP8BW_ERR_ALIAS;
+    for (int o2 = o + 1; o2 < count; ++o2)
+      if (overlap(outs[o], outs[o2])) return FP8BW_ERR_ALIAS;
+  }
+  DeviceInfo dev;
+  int st = current_device_info(&dev);
+  if (st != FP8BW_OK) return st;
+  const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (count == 0) return FP8BW_OK;
+  if (pow2 || jobs[0].m == 0) {
+    // one launch (or, for an empty contraction, one fill) per problem
+    for (int i = 0; i < count; ++i) {
+      st = run_gemm(ps[i], cs);
+      if (st != FP8BW_OK) return st;
+    }
+    return FP8BW_OK;
+  }
+  GemmProblem live[gemm::kMaxGemmJobs];
+  int nlive = 0;
+  for (int i = 0; i < count; ++i)
+    if (ps[i].mo > 0 && ps[i].no > 0) live[nlive++] = ps[i];
+  if (nlive == 0) return FP8BW_OK;
+  if (out_mode == kOutF32)
+    return launch_gemm_pair<GEMM_BN_VEC, true, false, kOutF32, gemm::kMaxGemmJobs>(live, nlive,
+                                                                                  dev, cs);
+  if (out_mode == kOutF32Add)
+    return launch_gemm_pair<GEMM_BN_VEC, true, false, kOutF32Add, gemm::kMaxGemmJobs>(
+        live, nlive, dev, cs);
+  return launch_gemm_pair<GEMM_BN_VEC, true, false, kOutBf16, gemm::kMaxGemmJobs>(live, nlive,
+                                                                                 dev, cs);
 }
 
 }  // namespace
@@ -796,6 +881,24 @@ int fp8bw_gemm_wgrad_f32_pow2(const uint8_t* qdy_t, const float* sdy_t, const ui
                               int accumulate, void* stream) {
   return wgrad_common(qdy_t, sdy_t, qx_t, sx_t, m, n, k, dw,
                       accumulate ? kOutF32Add : kOutF32, true, stream);
+}
+
+int fp8bw_gemm_wgrad_batch(const fp8bw_wgrad_job* jobs, int count, void* stream) {
+  return wgrad_batch(jobs, count, kOutBf16, false, stream);
+}
+
+int fp8bw_gemm_wgrad_batch_pow2(const fp8bw_wgrad_job* jobs, int count, void* stream) {
+  return wgrad_batch(jobs, count, kOutBf16, true, stream);
+}
+
+int fp8bw_gemm_wgrad_f32_batch(const fp8bw_wgrad_job* jobs, int count, int accumulate,
+                               void* stream) {
+  return wgrad_batch(jobs, count, accumulate ? kOutF32Add : kOutF32, false, stream);
+}
+
+int fp8bw_gemm_wgrad_f32_batch_pow2(const fp8bw_wgrad_job* jobs, int count, int accumulate,
+                                    void* stream) {
+  return wgrad_batch(jobs, count, accumulate ? kOutF32Add : kOutF32, true, stream);
 }
 
 int fp8bw_selftest_wait_timeout(int64_t limit_ns, void* stream) {

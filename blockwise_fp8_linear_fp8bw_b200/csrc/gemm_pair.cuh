@@ -101,6 +101,29 @@ struct Args {
   float* st_out;              // kOutBf16QQ: their scales [ceil(mo/128)][no]
 };
 
+// One launch can compute up to kMaxGemmJobs independent problems of the same
+// form (the weight gradients of several linears, say): their pair tiles are
+// numbered one problem after another, and every role finds a tile's problem
+// from the cumulative tile counts. All jobs have the same contraction length.
+// The tensor maps are __grid_constant__ (the TMA unit reads them in place);
+// the arguments are a plain by-value parameter. Both are read with constant
+// indices only (a chain of selects, or one call site per job for a tensor-map
+// address): measured by ptxas, arguments in a __grid_constant__ struct or a
+// tensor-map address computed from the job index cost the promotion warps
+// enough registers to spill.
+constexpr int kMaxGemmJobs = 4;
+template <int NJ>
+struct PairMaps {
+  CUtensorMap a[NJ];
+  CUtensorMap b[NJ];
+  CUtensorMap out[NJ];
+};
+template <int NJ>
+struct PairArgs {
+  Args job[NJ];
+  int tile_end[NJ];           // pair tiles of jobs 0..j; unused jobs repeat the total
+};
+
 __device__ __forceinline__ void setmaxnreg_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
 }
@@ -147,12 +170,31 @@ struct PairLayout {
   static_assert(kAlloc <= 227 * 1024, "shared memory budget");
 };
 
-template <int BN_, bool VEC_B, bool B_MN, int OUT = kOutBf16>
+template <int BN_, bool VEC_B, bool B_MN, int OUT = kOutBf16, int NJ = 1>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    blockwise_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
-                               const __grid_constant__ CUtensorMap tm_b,
-                               const __grid_constant__ CUtensorMap tm_out,
-                               const Args g) {
+    blockwise_gemm_pair_kernel(const __grid_constant__ PairMaps<NJ> maps,
+                               const PairArgs<NJ> pa) {
+  static_assert(NJ >= 1 && NJ <= kMaxGemmJobs, "job count");
+// Member f of job j's arguments (or of the tile counts), chosen among
+// constant-index reads of the parameter.
+#define FP8BW_PICK(j, f)                                        \
+  (NJ == 1 || (j) == 0 ? pa.f[0]                                \
+   : (j) == 1          ? pa.f[NJ > 1 ? 1 : 0]                   \
+   : (j) == 2          ? pa.f[NJ > 2 ? 2 : 0]                   \
+                       : pa.f[NJ > 3 ? 3 : 0])
+#define FP8BW_ARG(j, f)                                         \
+  (NJ == 1 || (j) == 0 ? pa.job[0].f                            \
+   : (j) == 1          ? pa.job[NJ > 1 ? 1 : 0].f               \
+   : (j) == 2          ? pa.job[NJ > 2 ? 2 : 0].f               \
+                       : pa.job[NJ > 3 ? 3 : 0].f)
+// The job of pair tile `tile` and the tile's index within that job.
+#define FP8BW_FIND_JOB(tile, job, lt)                           \
+  int job = 0, lt = (tile);                                     \
+  if constexpr (NJ > 1) {                                       \
+    _Pragma("unroll") for (int i_ = 0; i_ + 1 < NJ; ++i_)       \
+      job += lt >= FP8BW_PICK(i_, tile_end) ? 1 : 0;            \
+    if (job > 0) lt -= FP8BW_PICK(job - 1, tile_end);           \
+  }
   using L = PairLayout<BN_, VEC_B>;
   constexpr int BN = L::BN;
   constexpr int kScaleStages = L::kScaleStages;
@@ -207,9 +249,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tm_a);
-    prefetch_tmap(&tm_b);
-    prefetch_tmap(&tm_out);
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+      if (j > 0 && FP8BW_PICK(j - 1, tile_end) == FP8BW_PICK(j, tile_end)) continue;  // unused
+      prefetch_tmap(&maps.a[j]);
+      prefetch_tmap(&maps.b[j]);
+      prefetch_tmap(&maps.out[j]);
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(smem_u32(const_cast<uint32_t*>(tmem_slot)), L::kTmemCols);
@@ -225,8 +271,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   launch_dependents();
   grid_dependency_wait();
 
-  const int num_tiles = g.tiles_m * g.tiles_n;       // pair tiles (256 x 256)
-  const int C = g.chunks;
+  const int num_tiles = pa.tile_end[NJ - 1];         // pair tiles of all jobs
+  const int C = pa.job[0].chunks;                    // the same for every job
   const int cluster_id = blockIdx.x >> 1;
   const int num_clusters = gridDim.x >> 1;
 
@@ -244,7 +290,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int tile = cluster_id; ok && tile < num_tiles; tile += num_clusters) {
-        const int tm = tile / g.tiles_n, tn = tile % g.tiles_n;
+        FP8BW_FIND_JOB(tile, job, lt)
+        const int tm = lt / FP8BW_ARG(job, tiles_n), tn = lt % FP8BW_ARG(job, tiles_n);
         const int a_row = tm * (2 * BM) + static_cast<int>(rank) * BM;
         const int b_row = tn * BN + static_cast<int>(rank) * (BN / 2);
         for (int c = 0; c < C; ++c, ++it) {
@@ -258,11 +305,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint32_t b_dst = a_dst + L::kABytes;
           const uint32_t fbar = full_leader0 + 8u * s;
           if (leader) mbar_arrive_expect_tx(full_bar(s), 2 * L::kStageBytes);
-          tma_load_2d_pair(a_dst, &tm_a, fbar, c * BK, a_row);
+          tma_load_2d_pair(a_dst, &maps.a[job], fbar, c * BK, a_row);
           if constexpr (B_MN)
-            tma_load_2d_pair(b_dst, &tm_b, fbar, b_row, c * BK);
+            tma_load_2d_pair(b_dst, &maps.b[job], fbar, b_row, c * BK);
           else
-            tma_load_2d_pair(b_dst, &tm_b, fbar, c * BK, b_row);
+            tma_load_2d_pair(b_dst, &maps.b[job], fbar, c * BK, b_row);
         }
       }
       if (!ok && leader) {
@@ -332,10 +379,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int cc = static_cast<int>(fi - k * C);
       const int64_t t = cluster_id + k * num_clusters;
       if (t < num_tiles) {
-        const int jb0 = static_cast<int>(t % g.tiles_n) * (BN / 128);
-        p0 = __ldg(g.sb + jb0 * g.sbj + static_cast<int64_t>(cc) * g.sbc);
-        if (BN > 128 && jb0 + 1 < g.nblk)
-          p1 = __ldg(g.sb + (jb0 + 1) * g.sbj + static_cast<int64_t>(cc) * g.sbc);
+        FP8BW_FIND_JOB(static_cast<int>(t), tj, tl)
+        const int jb0 = (tl % FP8BW_ARG(tj, tiles_n)) * (BN / 128);
+        p0 = __ldg(FP8BW_ARG(tj, sb) + jb0 * FP8BW_ARG(tj, sbj) +
+                   static_cast<int64_t>(cc) * FP8BW_ARG(tj, sbc));
+        if (BN > 128 && jb0 + 1 < FP8BW_ARG(tj, nblk))
+          p1 = __ldg(FP8BW_ARG(tj, sb) + (jb0 + 1) * FP8BW_ARG(tj, sbj) +
+                     static_cast<int64_t>(cc) * FP8BW_ARG(tj, sbc));
       }
     };
     float cur0 = 0.0f, cur1 = 0.0f, nxt0 = 0.0f, nxt1 = 0.0f;
@@ -346,11 +396,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint32_t sit = 0;
     bool ok = true;
     for (int tile = cluster_id; ok && tile < num_tiles; tile += num_clusters) {
-      const int tm = tile / g.tiles_n, tn = tile % g.tiles_n;
+      FP8BW_FIND_JOB(tile, job, lt)
+      const int tm = lt / FP8BW_ARG(job, tiles_n), tn = lt % FP8BW_ARG(job, tiles_n);
       const int m0 = tm * (2 * BM) + static_cast<int>(rank) * BM, n0 = tn * BN;
-      const int rows_here = max(0, min(BM, g.mo - m0));
+      const int rows_here = max(0, min(BM, FP8BW_ARG(job, mo) - m0));
       const uint32_t a_bytes = static_cast<uint32_t>(rows_here) * 4u;
-      const uint32_t b_bytes = VEC_B ? static_cast<uint32_t>(min(BN, g.no - n0)) * 4u : 0u;
+      const uint32_t b_bytes = VEC_B ? static_cast<uint32_t>(min(BN, FP8BW_ARG(job, no) - n0)) * 4u : 0u;
       for (int c = 0; c < C; ++c, ++sit) {
         if constexpr (!VEC_B) {
           if ((sit & 31u) == 0 && sit > 0) {
@@ -375,10 +426,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
             mbar_arrive_expect_tx(sfull_bar(ss), a_bytes + b_bytes);
             if (a_bytes > 0)
-              bulk_load(slot_u, g.sa + static_cast<int64_t>(c) * g.mo + m0, a_bytes,
+              bulk_load(slot_u, FP8BW_ARG(job, sa) + static_cast<int64_t>(c) * FP8BW_ARG(job, mo) + m0, a_bytes,
                         sfull_bar(ss));
             if constexpr (VEC_B)
-              bulk_load(slot_u + L::kSaBytes, g.sb + static_cast<int64_t>(c) * g.no + n0,
+              bulk_load(slot_u + L::kSaBytes, FP8BW_ARG(job, sb) + static_cast<int64_t>(c) * FP8BW_ARG(job, no) + n0,
                         b_bytes, sfull_bar(ss));
           }
         }
@@ -413,7 +464,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint32_t box_seq = 0;         // kOutBf16QQ: boxes this warp has quantised
     bool ok = true, store_pending = false;
     for (int tile = cluster_id; ok && tile < num_tiles; tile += num_clusters) {
-      const int tm = tile / g.tiles_n, tn = tile % g.tiles_n;
       uint64_t acc2[kHalf / 2];   // fp32 accumulator pairs (columns 2i, 2i+1)
 #pragma unroll
       for (int j = 0; j < kHalf / 2; ++j) acc2[j] = 0ull;
@@ -516,6 +566,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       float acc[kHalf];
 #pragma unroll
       for (int j = 0; j < kHalf / 2; ++j) unpack2(acc2[j], acc[2 * j], acc[2 * j + 1]);
+      // the tile's job, looked up after the chunk loop (nothing of it is live
+      // during it)
+      FP8BW_FIND_JOB(tile, job, lt)
+      const int mo_j = FP8BW_ARG(job, mo), no_j = FP8BW_ARG(job, no);
+      const int tm = lt / FP8BW_ARG(job, tiles_n), tn = lt % FP8BW_ARG(job, tiles_n);
 
       const int y0 = tm * (2 * BM) + static_cast<int>(rank) * BM + q * 32;
       const int x0 = tn * BN + h * kHalf;
@@ -531,7 +586,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         float sc;
         group_scale(max_halves(mx), qscale, sc);
         const int grow = y0 + lane;
-        if (grow < g.mo && x0 < g.no) g.s_out[static_cast<int64_t>(x0 / 128) * g.mo + grow] = sc;
+        if (grow < mo_j && x0 < no_j) FP8BW_ARG(job, s_out)[static_cast<int64_t>(x0 / 128) * mo_j + grow] = sc;
       }
       // One 2 KB staging box per warp: 32 rows of 64 bytes (32 bf16 or 16
       // fp32 columns), 64-byte swizzle (16-byte unit j of row r at j ^ (r/2 % 4)).
@@ -541,8 +596,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // kOutBf16QQ: the four warps of this column half exchange column
         // maxima for every box that has columns in range, so a warp whose
         // rows are all past the end still takes part (it stores nothing).
-        if (x0 + gi * kBoxCols >= g.no) continue;
-        if (OUT != kOutBf16QQ && y0 >= g.mo) continue;
+        if (x0 + gi * kBoxCols >= no_j) continue;
+        if (OUT != kOutBf16QQ && y0 >= mo_j) continue;
         // the box that used this staging buffer kOutBoxes stores ago must
         // have been read by its TMA store
         const uint32_t stage_box = stage_out + (out_seq % L::kOutBoxes) * L::kOutWarpBytes;
@@ -613,10 +668,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           if constexpr (out_quant_rows(OUT)) {
             const int grow = y0 + lane;
-            if (grow < g.mo) {
-              uint8_t* dst = g.q_out + static_cast<int64_t>(grow) * g.no + x0 + gi * 32;
+            if (grow < mo_j) {
+              uint8_t* dst = FP8BW_ARG(job, q_out) + static_cast<int64_t>(grow) * no_j + x0 + gi * 32;
               *reinterpret_cast<uint4*>(dst) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-              if (x0 + gi * 32 + 16 < g.no)
+              if (x0 + gi * 32 + 16 < no_j)
                 *reinterpret_cast<uint4*>(dst + 16) =
                     make_uint4(codes[4], codes[5], codes[6], codes[7]);
             }
@@ -665,8 +720,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             group_scale(amax, cqs, csc);
             const int col = x0 + gi * 32 + lane;
             const int tg = tm * 2 + static_cast<int>(rank);     // token group
-            if (col < g.no) {
-              if (q == 0 && tg * 128 < g.mo) g.st_out[static_cast<int64_t>(tg) * g.no + col] = csc;
+            if (col < no_j) {
+              if (q == 0 && tg * 128 < mo_j) FP8BW_ARG(job, st_out)[static_cast<int64_t>(tg) * no_j + col] = csc;
               uint32_t cc[8];
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
@@ -675,21 +730,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 scale_pair(cv[2 * i + 1], cqs, t[2], t[3]);
                 cc[i] = e4m3x2(t[0], t[1]) | (e4m3x2(t[2], t[3]) << 16);
               }
-              uint8_t* dst = g.qt_out + static_cast<int64_t>(col) * g.mo + y0;
-              if (y0 < g.mo) *reinterpret_cast<uint4*>(dst) = make_uint4(cc[0], cc[1], cc[2], cc[3]);
-              if (y0 + 16 < g.mo)
+              uint8_t* dst = FP8BW_ARG(job, qt_out) + static_cast<int64_t>(col) * mo_j + y0;
+              if (y0 < mo_j) *reinterpret_cast<uint4*>(dst) = make_uint4(cc[0], cc[1], cc[2], cc[3]);
+              if (y0 + 16 < mo_j)
                 *reinterpret_cast<uint4*>(dst + 16) = make_uint4(cc[4], cc[5], cc[6], cc[7]);
             }
-            if (y0 >= g.mo) continue;       // nothing of this warp's box to store
+            if (y0 >= mo_j) continue;       // nothing of this warp's box to store
           }
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          if constexpr (OUT == kOutF32Add)
-            tma_reduce_add_2d(&tm_out, stage_box, x0 + gi * kBoxCols, y0);
-          else
-            tma_store_2d(&tm_out, stage_box, x0 + gi * kBoxCols, y0);
+          const int bx = x0 + gi * kBoxCols;
+          auto issue = [&](const CUtensorMap* map) {
+            if constexpr (OUT == kOutF32Add)
+              tma_reduce_add_2d(map, stage_box, bx, y0);
+            else
+              tma_store_2d(map, stage_box, bx, y0);
+          };
+          // one call site per job, each with a constant tensor-map address
+          if (NJ == 1 || job == 0) issue(&maps.out[0]);
+          else if (job == 1) issue(&maps.out[NJ > 1 ? 1 : 0]);
+          else if (job == 2) issue(&maps.out[NJ > 2 ? 2 : 0]);
+          else issue(&maps.out[NJ > 3 ? 3 : 0]);
           bulk_commit_group();
         }
         store_pending = true;
@@ -708,6 +771,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tmem_dealloc_pair(tmem_base, L::kTmemCols);
   }
 }
+#undef FP8BW_FIND_JOB
+#undef FP8BW_ARG
+#undef FP8BW_PICK
 
 }  // namespace gemm
 }  // namespace fp8bw

@@ -222,6 +222,47 @@ def fp8bw_gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, dw, accumulate=False,
           _ptr(dw), 1 if accumulate else 0)
 
 
+def _wgrad_jobs(jobs, dtype):
+    """ctypes array of fp8bw_wgrad_job from (qdy_t, sdy_t, qx_t, sx_t, dw)
+    tuples, and the tensors it points into."""
+    arr = (_native.WgradJob * len(jobs))()
+    tensors = []
+    for i, (qdy_t, sdy_t, qx_t, sx_t, dw) in enumerate(jobs):
+        n, m = qdy_t.shape
+        k = qx_t.shape[0]
+        _expect(qdy_t, torch.uint8, (n, m), "jobs[%d].qdy_t" % i)
+        _expect(qx_t, torch.uint8, (k, m), "jobs[%d].qx_t" % i)
+        _expect(sdy_t, torch.float32, (_cdiv(m, 128), n), "jobs[%d].sdy_t" % i)
+        _expect(sx_t, torch.float32, (_cdiv(m, 128), k), "jobs[%d].sx_t" % i)
+        _expect(dw, dtype, (n, k), "jobs[%d].dw" % i)
+        arr[i] = _native.WgradJob(_ptr(qdy_t), _ptr(sdy_t), _ptr(qx_t),
+                                  _ptr(sx_t), m, n, k, _ptr(dw))
+        tensors += [qdy_t, sdy_t, qx_t, sx_t, dw]
+    return arr, tensors
+
+
+def fp8bw_gemm_wgrad_batch(jobs, stream=None, pow2=False):
+    """Up to 4 weight gradients over the same tokens in one launch: each job
+    (qdy_t, sdy_t, qx_t, sx_t, dw) is fp8bw_gemm_wgrad of its arguments (bf16
+    dw)."""
+    if not jobs:
+        return
+    arr, tensors = _wgrad_jobs(jobs, torch.bfloat16)
+    _call(_fn("fp8bw_gemm_wgrad_batch", pow2), tensors, stream,
+          ctypes.cast(arr, ctypes.c_void_p), len(jobs))
+
+
+def fp8bw_gemm_wgrad_f32_batch(jobs, accumulate=False, stream=None,
+                               pow2=False):
+    """The fp32-dW form of fp8bw_gemm_wgrad_batch (each job as
+    fp8bw_gemm_wgrad_f32, the same `accumulate` for all)."""
+    if not jobs:
+        return
+    arr, tensors = _wgrad_jobs(jobs, torch.float32)
+    _call(_fn("fp8bw_gemm_wgrad_f32_batch", pow2), tensors, stream,
+          ctypes.cast(arr, ctypes.c_void_p), len(jobs), 1 if accumulate else 0)
+
+
 def fp8bw_gemm_fprop_quant(qx, sx, qw, sw, y, qy, sy, stream=None):
     m, k = qx.shape
     n = qw.shape[0]
@@ -398,6 +439,31 @@ def gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, main_grad=None, stream=None,
                      device=qdy_t.device)
     fp8bw_gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, dw, False, stream, pow2=pow2)
     return dw
+
+
+def gemm_wgrad_batch(operands, stream=None, pow2=False):
+    """-> [bf16 dW] for each (qdy_t, sdy_t, qx_t, sx_t) in `operands` (same
+    token count), computed in one launch."""
+    dws = [torch.empty((o[0].shape[0], o[2].shape[0]), dtype=torch.bfloat16,
+                       device=o[0].device) for o in operands]
+    fp8bw_gemm_wgrad_batch([tuple(o) + (dw,) for o, dw in zip(operands, dws)],
+                           stream, pow2=pow2)
+    return dws
+
+
+def gemm_wgrad_f32_batch(operands, main_grads=None, stream=None, pow2=False):
+    """fp32 dWs of fp8bw_gemm_wgrad_f32_batch; with `main_grads` given (one
+    fp32 tensor per job), each dW is added into its main-grad in place and the
+    main-grads are returned."""
+    if main_grads is not None:
+        fp8bw_gemm_wgrad_f32_batch([tuple(o) + (g,) for o, g in zip(operands, main_grads)],
+                                   True, stream, pow2=pow2)
+        return list(main_grads)
+    dws = [torch.empty((o[0].shape[0], o[2].shape[0]), dtype=torch.float32,
+                       device=o[0].device) for o in operands]
+    fp8bw_gemm_wgrad_f32_batch([tuple(o) + (dw,) for o, dw in zip(operands, dws)],
+                               False, stream, pow2=pow2)
+    return dws
 
 
 def gemm_fprop_quant(qx, sx, qw, sw, stream=None):

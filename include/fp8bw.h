@@ -189,6 +189,37 @@ int fp8bw_gemm_wgrad_f32(const uint8_t* qdy_t, const float* sdy_t,
                          int64_t n, int64_t k, float* dw, int accumulate,
                          void* stream);
 
+/* Several weight gradients in one launch (the linears of a layer, whose
+ * backward passes all contract over the same tokens): each job is exactly
+ * what fp8bw_gemm_wgrad (bf16 dW) or fp8bw_gemm_wgrad_f32 (fp32 dW, stored
+ * or, with accumulate != 0, added into dw) computes for its arguments; the
+ * jobs' output tiles share one persistent grid, so the last wave of one
+ * problem is filled with tiles of the next.
+ *   jobs       : HOST array of `count` job descriptions (read during the call
+ *                only); pointers are device pointers with the layouts of
+ *                fp8bw_gemm_wgrad; dw is bf16 [n, k] for
+ *                fp8bw_gemm_wgrad_batch, fp32 [n, k] for the _f32 form.
+ *   count      : 0..4 (0 is a no-op; more is FP8BW_ERR_SHAPE).
+ *   accumulate : the same for every job.
+ * Errors: a job's own checks as the single-problem call; all jobs must have
+ * the same m (FP8BW_ERR_SHAPE); no dw may overlap any job's input or another
+ * dw (FP8BW_ERR_ALIAS). Nothing is launched when a check fails.
+ * Source: paperlayer.ai summary, Appendix C, "FP8 implementation pipeline"
+ * (the weight-gradient GEMM of each linear). */
+typedef struct fp8bw_wgrad_job {
+    const uint8_t* qdy_t;   /* col-wise quantised dY: codes [n, m]           */
+    const float* sdy_t;     /*   scales [ceil(m/128)][n]                     */
+    const uint8_t* qx_t;    /* col-wise quantised X: codes [k, m]            */
+    const float* sx_t;      /*   scales [ceil(m/128)][k]                     */
+    int64_t m, n, k;
+    void* dw;               /* bf16 or fp32 [n, k], per the entry point      */
+} fp8bw_wgrad_job;
+
+int fp8bw_gemm_wgrad_batch(const fp8bw_wgrad_job* jobs, int count,
+                           void* stream);
+int fp8bw_gemm_wgrad_f32_batch(const fp8bw_wgrad_job* jobs, int count,
+                               int accumulate, void* stream);
+
 /* fprop / dgrad that also quantise their own bf16 output row-wise, for a
  * linear that consumes it next: the same y (dx) as fp8bw_gemm_fprop
  * (fp8bw_gemm_dgrad), plus exactly what fp8bw_quantize_rowwise would write
@@ -293,6 +324,12 @@ int fp8bw_gemm_wgrad_f32_pow2(const uint8_t* qdy_t, const float* sdy_t,
                               const uint8_t* qx_t, const float* sx_t,
                               int64_t m, int64_t n, int64_t k, float* dw,
                               int accumulate, void* stream);
+/* The batched forms (one launch per job: the power-of-two kernel takes one
+ * problem at a time); checks and errors as fp8bw_gemm_wgrad_batch. */
+int fp8bw_gemm_wgrad_batch_pow2(const fp8bw_wgrad_job* jobs, int count,
+                                void* stream);
+int fp8bw_gemm_wgrad_f32_batch_pow2(const fp8bw_wgrad_job* jobs, int count,
+                                    int accumulate, void* stream);
 
 /* Synchronises `stream`, then returns FP8BW_ERR_DEVICE_TIMEOUT if any kernel
  * of this library on the current device recorded an expired wait since the

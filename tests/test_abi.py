@@ -37,14 +37,14 @@ def lib():
 
 def test_every_declared_symbol_is_exported(lib):
     names = declared_functions()
-    assert len(names) == 24
+    assert len(names) == 28
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(_native.SIGNATURES)
 
 
 def test_status_strings_and_version(lib):
-    assert lib.fp8bw_version() == 107
+    assert lib.fp8bw_version() == 108
     for st in (OK, E_NULL, E_SHAPE, E_ALIGN, E_DEVICE, E_LAUNCH, E_TIMEOUT,
                E_CUDA, E_ALIAS, E_SCALE):
         s = lib.fp8bw_status_string(st).decode()
@@ -181,10 +181,48 @@ def test_weight_block_batch_checks(lib):
     assert lib.fp8bw_quantize_weight_block_batch(p, 2, None) == E_ALIAS
 
 
+def _wjobs(*specs):
+    arr = (_native.WgradJob * max(1, len(specs)))()
+    for i, sp in enumerate(specs):
+        arr[i] = _native.WgradJob(*sp)
+    return ctypes.cast(arr, ctypes.c_void_p), arr
+
+
+def test_wgrad_batch_checks(lib):
+    M = 0x1000000
+    # qdy_t, sdy_t, qx_t, sx_t, m, n, k, dw
+    ok1 = (A, B, C, D, 256, 128, 256, E)
+    ok2 = (A + M, B + M, C + M, D + M, 256, 256, 128, E + M)
+    p, keep = _wjobs(ok1, ok2)
+    for fn in (lib.fp8bw_gemm_wgrad_batch, lib.fp8bw_gemm_wgrad_batch_pow2):
+        assert fn(p, 5, None) == E_SHAPE
+        assert fn(p, -1, None) == E_SHAPE
+        assert fn(None, 2, None) == E_NULL
+    assert lib.fp8bw_gemm_wgrad_f32_batch(p, 5, 1, None) == E_SHAPE
+    assert lib.fp8bw_gemm_wgrad_f32_batch_pow2(None, 1, 0, None) == E_NULL
+    # different token counts
+    p, keep = _wjobs(ok1, ok2[:4] + (384,) + ok2[5:])
+    assert lib.fp8bw_gemm_wgrad_batch(p, 2, None) == E_SHAPE
+    # a job's own checks: ragged size, null operand, misaligned dW
+    p, keep = _wjobs(ok1, ok2[:5] + (100,) + ok2[6:])
+    assert lib.fp8bw_gemm_wgrad_batch(p, 2, None) == E_SHAPE
+    p, keep = _wjobs(ok1, (None,) + ok2[1:])
+    assert lib.fp8bw_gemm_wgrad_f32_batch(p, 2, 0, None) == E_NULL
+    p, keep = _wjobs(ok1, ok2[:7] + (E + M + 8,))
+    assert lib.fp8bw_gemm_wgrad_batch(p, 2, None) == E_ALIGN
+    # job 2's dW on top of job 1's operand, and two jobs sharing a dW
+    p, keep = _wjobs(ok1, ok2[:7] + (C + 64,))
+    assert lib.fp8bw_gemm_wgrad_batch(p, 2, None) == E_ALIAS
+    p, keep = _wjobs(ok1, ok2[:7] + (E + 1024,))
+    assert lib.fp8bw_gemm_wgrad_f32_batch(p, 2, 1, None) == E_ALIAS
+
+
 @pytest.mark.skipif(
     __import__("torch").cuda.is_available(),
     reason="checks the no-device path; on a GPU host the call would launch")
 def test_valid_call_without_device_reports_device_error(lib):
+    p, keep = _wjobs((A, B, C, D, 256, 128, 256, E))
+    assert lib.fp8bw_gemm_wgrad_batch(p, 1, None) == E_DEVICE
     p, keep = _jobs((A, 256, 128, B, C, D))
     assert lib.fp8bw_quantize_weight_block_batch(p, 1, None) == E_DEVICE
     assert lib.fp8bw_quantize_rowwise(A, 128, 128, B, C, None) == E_DEVICE

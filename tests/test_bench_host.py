@@ -88,8 +88,10 @@ class _FakeLinear:
 
     def ops(self, o, stream, pow2=False):
         return [("quant_rowcol", 1e6, lambda: None),
-                ("gemm_block_scaled", 1e9, lambda: None),
-                ("gemm_vector_scaled", 1e9, lambda: None)]
+                ("gemm_block_scaled", 1e9, lambda: None)]
+
+    def wgrad_job(self):
+        return (self.qdy_t, self.sdy_t, self.qx_t, self.sx_t, None)
 
 
 def test_next_rows_host_logic_with_stubbed_device(monkeypatch):
@@ -112,8 +114,10 @@ def test_next_rows_host_logic_with_stubbed_device(monkeypatch):
     assert lib.calls["fp8bw_gemm_fprop_quant_rowcol"] == \
         lib.calls["fp8bw_gemm_dgrad_quant_rowcol"]
     assert ("%d-layer" % bench.LAYERS) in out["pow2_step"]["what"]
-    assert out["wgrad_f32_accumulate"]["launches"] == 5 * len(bufs)
-    assert lib.calls["fp8bw_gemm_wgrad_f32"] == 2 * (3 + 5)
+    assert out["wgrad_f32_accumulate"]["launches"] == 5
+    assert lib.calls["fp8bw_gemm_wgrad_f32_batch"] == 3 + 5
+    # the power-of-two step: one batched wgrad per layer
+    assert lib.calls["fp8bw_gemm_wgrad_batch"] == 3 * bench.LAYERS + 3 * bench.LAYERS
     # fprop runs in the row-wise and the row + column comparison alike
     assert 2 * lib.calls["fp8bw_gemm_fprop_quant"] == lib.calls["fp8bw_gemm_fprop"]
     assert set(out["pow2_step"]["breakdown"]) == {
