@@ -53,19 +53,20 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
                   "bf16_tflops_sustained": 1400.0}
 FP8_OVER_BF16 = 2.0   # nominal dense FP8 / BF16 tensor throughput (4.5 / 2.25)
 
-# DRAM bytes (read + write) per launch of each kernel, averaged over the 672
-# launches of one step, from one ncu capture (gpu__time_duration.sum,
-# dram__bytes_read.sum, dram__bytes_write.sum; profiles/
-# launches_stack28_m16384.md). Valid only for the kernel sources they were
+# DRAM bytes (read + write) per launch of each kernel kind, from one ncu
+# capture (gpu__time_duration.sum, dram__bytes_read.sum, dram__bytes_write.sum)
+# of a one-layer step: its 18 launches are those every layer of the full step
+# repeats at the same sizes, so their per-kind average is the full step's
+# (profiles/dram_layer_m16384.md). Valid only for the kernel sources they were
 # taken on: KERNEL_FINGERPRINT is a hash of csrc/*.cu[h] at that time, and the
 # numbers are reported as null once the sources differ.
 NCU_TRAFFIC_PER_LAUNCH = {
-    "gemm_block_scaled": 183655835,
-    "gemm_vector_scaled": 253264658,
-    "quant_rowcol": 217274385,
-    "quant_weight_block": 25456937,
+    "gemm_block_scaled": 184835040,
+    "gemm_vector_scaled": 1189339648,
+    "quant_rowcol": 217172992,
+    "quant_weight_block": 147285760,
 }
-KERNEL_FINGERPRINT = "9e8dd45068db543e"
+KERNEL_FINGERPRINT = "3a36cf32c960d0ce"
 
 
 def kernel_fingerprint():
