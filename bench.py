@@ -913,7 +913,7 @@ def result_line(args, world, res):
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        sample = OracleSample(tokens=256)
+        sample = OracleSample(tokens=1024)
         t0 = time.perf_counter()
         sample.run()
         dt = time.perf_counter() - t0
