@@ -94,7 +94,7 @@ struct Args {
   const float* sb;            // vector: [chunks][no]; block: sb[jb*sbj + c*sbc]
   int64_t sbj, sbc;
   int nblk;                   // number of 128-wide output column blocks
-  void* out;                  // [mo][no], bf16 or fp32 (written through tm_out)
+  void* out;                  // [mo][no], bf16 or fp32 (written through the job's output tensor map)
   uint8_t* q_out;             // kOutBf16Q(Q): codes [mo][no]
   float* s_out;               // kOutBf16Q(Q): scales [ceil(no/128)][mo]
   uint8_t* qt_out;            // kOutBf16QQ: transposed column-wise codes [no][mo]
