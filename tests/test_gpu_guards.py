@@ -182,3 +182,36 @@ def test_weight_block_batch_writes_exactly_its_outputs(pow2):
     for w, q, s, q_t in zip(ws, qs, ss, qts):
         rq, rs, rq_t = ops.quantize_weight_block(w, pow2=pow2)
         assert _eq(q, rq) and _eq(s, rs) and _eq(q_t, rq_t)
+
+
+@pytest.mark.parametrize("pow2", [False, True])
+def test_wgrad_batch_writes_exactly_its_outputs(pow2):
+    """Four wgrad jobs of ragged shapes over the same tokens in one call: bf16
+    dW, fp32 dW and the fp32 add into a main-grad, each in its own guarded
+    buffer."""
+    import torch
+    ops = _ops()
+    m = 400
+    shapes = [(272, 400), (16, 16), (1040, 144), (384, 1296)]   # (n, k)
+    operands = []
+    for i, (n, k) in enumerate(shapes):
+        dy = bf16_np_to_torch(S.bf16_normal((m, n), 0, 1500 + 2 * i, **S.DY_DIST))
+        x = bf16_np_to_torch(S.bf16_normal((m, k), 0, 1501 + 2 * i, **S.X_DIST))
+        operands.append(ops.quantize_colwise(dy, pow2=pow2) + ops.quantize_colwise(x, pow2=pow2))
+    g = Guarded()
+    dws = [g.make(sh, torch.bfloat16) for sh in shapes]
+    dw32 = [g.make(sh, torch.float32) for sh in shapes]
+    acc32 = [g.make(sh, torch.float32) for sh in shapes]
+    for a in acc32:
+        a.zero_()
+    ops.fp8bw_gemm_wgrad_batch([tuple(o) + (d,) for o, d in zip(operands, dws)], pow2=pow2)
+    ops.fp8bw_gemm_wgrad_f32_batch([tuple(o) + (d,) for o, d in zip(operands, dw32)],
+                                   pow2=pow2)
+    ops.fp8bw_gemm_wgrad_f32_batch([tuple(o) + (d,) for o, d in zip(operands, acc32)],
+                                   accumulate=True, pow2=pow2)
+    ops.fp8bw_check_device_error()
+    g.check("batched wgrad")
+    for o, d, d32, a32 in zip(operands, dws, dw32, acc32):
+        assert _eq(d, ops.gemm_wgrad(*o, pow2=pow2))
+        ref32 = ops.gemm_wgrad_f32(*o, pow2=pow2)
+        assert _eq(d32, ref32) and _eq(a32, ref32)

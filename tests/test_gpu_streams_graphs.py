@@ -1,7 +1,7 @@
 """Calls are asynchronous on the stream they are given and keep no state
-between calls (no shared scratch): two streams running the linear step at the
-same time give the serial results, and the whole step captured in a CUDA
-graph and replayed gives the eager results."""
+between calls (no shared scratch): two streams running the linear step (with
+a batched wgrad launch) at the same time give the serial results, and the
+whole step captured in a CUDA graph and replayed gives the eager results."""
 import pytest
 
 import synthetic as S
@@ -24,7 +24,10 @@ def _step(ops, x, w, dy, stream):
     qdy_t, sdy_t, qdy, sdy = ops.quantize_colwise(dy, with_rowwise=True, stream=stream)
     dx = ops.gemm_dgrad(qdy, sdy, qw_t, sw, stream=stream)
     dw = ops.gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t, stream=stream)
-    return y, dx, dw
+    # the batched form, with a second job of another shape (dW transposed)
+    dwb = ops.gemm_wgrad_batch([(qdy_t, sdy_t, qx_t, sx_t), (qx_t, sx_t, qdy_t, sdy_t)],
+                               stream=stream)
+    return (y, dx, dw, *dwb)
 
 
 def _same(a, b):
@@ -71,6 +74,7 @@ def test_step_in_a_cuda_graph():
     torch.cuda.synchronize()
     ops.fp8bw_check_device_error()
     assert _same(out, ref)
+    assert _same(out[3:4], out[2:3])     # the batch's first job is the single wgrad
     # new inputs copied into the captured buffers are picked up by a replay
     x2, w2, dy2 = _inputs(1005)
     ref2 = _step(ops, x2, w2, dy2, torch.cuda.current_stream())
