@@ -58,25 +58,32 @@ FP8_OVER_BF16 = 2.0   # nominal dense FP8 / BF16 tensor throughput (4.5 / 2.25)
 # of a one-layer step: its 18 launches are those every layer of the full step
 # repeats at the same sizes, so their per-kind average is the full step's
 # (profiles/dram_layer_m16384.md). Valid only for the kernel sources they were
-# taken on: KERNEL_FINGERPRINT is a hash of csrc/*.cu[h] at that time, and the
-# numbers are reported as null once the sources differ.
+# taken on: KERNEL_FINGERPRINT is kernel_fingerprint() of the sources at that
+# time, and the numbers are reported as null once the code differs.
 NCU_TRAFFIC_PER_LAUNCH = {
     "gemm_block_scaled": 184835040,
     "gemm_vector_scaled": 1189339648,
     "quant_rowcol": 217172992,
     "quant_weight_block": 147285760,
 }
-KERNEL_FINGERPRINT = "3a36cf32c960d0ce"
+KERNEL_FINGERPRINT = "37a8d0789a95e96b"
 
 
 def kernel_fingerprint():
+    """sha256 (first 16 hex digits) of csrc/*.cu[h] in name order, each with
+    its comments removed and whitespace collapsed: it changes with the code,
+    not with its comments."""
     import hashlib
+    import re
     h = hashlib.sha256()
     d = os.path.join(ROOT, "blockwise_fp8_linear_fp8bw_b200", "csrc")
     for f in sorted(os.listdir(d)):
         if f.endswith((".cu", ".cuh")):
-            with open(os.path.join(d, f), "rb") as fh:
-                h.update(fh.read())
+            with open(os.path.join(d, f)) as fh:
+                src = fh.read()
+            src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+            src = re.sub(r"//[^\n]*", " ", src)
+            h.update(" ".join(src.split()).encode())
     return h.hexdigest()[:16]
 
 
