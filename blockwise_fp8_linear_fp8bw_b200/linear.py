@@ -28,6 +28,9 @@ import torch
 
 from . import ops
 
+_WEIGHT_BATCH = 8     # weights per batched block-quantisation launch
+_WGRAD_BATCH = 4      # weight gradients per batched wgrad launch
+
 
 def _rows(t, k):
     if not t.is_cuda or t.dtype != torch.bfloat16:
@@ -111,24 +114,30 @@ class BlockwiseFp8ChainFunction(torch.autograd.Function):
     directly, each on the blockwise-FP8 path, with every intermediate
     quantisation fused into the GEMM that produces it.
 
-    Forward: each fprop but the last also writes the row-wise (next fprop)
-    and column-wise (next wgrad) codes of its bf16 output, so the next linear
-    reads codes instead of re-reading and re-quantising the activation.
+    Forward: the weights are block-quantised in batched launches (up to 8
+    per launch); each fprop but the last also writes the row-wise (next
+    fprop) and column-wise (next wgrad) codes of its bf16 output, so the next
+    linear reads codes instead of re-reading and re-quantising the activation.
     Backward: each dgrad but the first linear's does the same for the
-    gradient it produces, which is the previous linear's dY. The results are
+    gradient it produces, which is the previous linear's dY; the weight
+    gradients, which all contract over the same tokens, are deferred to the
+    end and computed in batched launches (up to 4 per launch). The results are
     those of the same linears run one by one (the fused codes are, bit for
-    bit, those of quantising the bf16 output)."""
+    bit, those of quantising the bf16 output, and a batched launch computes
+    what its jobs compute alone)."""
 
     @staticmethod
     def forward(ctx, x, *weights):
         k0 = weights[0].shape[1]
         h = _rows(x, k0)
         qx_t, sx_t, qx, sx = ops.quantize_colwise(h, with_rowwise=True)
+        ws = [_rows(w, w.shape[1]) for w in weights]
+        qws = []
+        for j in range(0, len(ws), _WEIGHT_BATCH):
+            qws += ops.quantize_weight_block_batch(ws[j:j + _WEIGHT_BATCH], transposed=True)
         saved = []
         y = None
-        for i, weight in enumerate(weights):
-            w = _rows(weight, weight.shape[1])
-            qw, sw, qw_t = ops.quantize_weight_block(w, transposed=True)
+        for i, (qw, sw, qw_t) in enumerate(qws):
             saved += [qx_t, sx_t, qw_t, sw]
             if i + 1 < len(weights):
                 y, qx, sx, qx_t, sx_t = ops.gemm_fprop_quant_rowcol(qx, sx, qw, sw)
@@ -148,22 +157,29 @@ class BlockwiseFp8ChainFunction(torch.autograd.Function):
         qdy_t, sdy_t, qdy, sdy = ops.quantize_colwise(dy2, with_rowwise=True)
         grads = [None] * len(weights)
         dx = None
+        to_main, to_grad = [], []      # deferred wgrads: (index, operands)
         for i in range(len(weights) - 1, -1, -1):
             qx_t, sx_t, qw_t, sw = saved[4 * i:4 * i + 4]
-            weight = weights[i]
             if ctx.needs_input_grad[1 + i]:
-                main = getattr(weight, "main_grad", None)
-                if main is not None:
-                    ops.gemm_wgrad_f32(qdy_t, sdy_t, qx_t, sx_t, main_grad=main)
+                job = (i, (qdy_t, sdy_t, qx_t, sx_t))
+                if getattr(weights[i], "main_grad", None) is not None:
+                    to_main.append(job)
                 else:
-                    dw = ops.gemm_wgrad(qdy_t, sdy_t, qx_t, sx_t)
-                    grads[i] = dw if dw.dtype == weight.dtype else dw.to(weight.dtype)
+                    to_grad.append(job)
             if i > 0:
                 _, qdy, sdy, qdy_t, sdy_t = ops.gemm_dgrad_quant_rowcol(
                     qdy, sdy, qw_t, sw, qw_is_transposed=True)
             elif ctx.needs_input_grad[0]:
                 dx = ops.gemm_dgrad(qdy, sdy, qw_t, sw,
                                     qw_is_transposed=True).reshape(ctx.x_shape)
+        for j in range(0, len(to_main), _WGRAD_BATCH):
+            part = to_main[j:j + _WGRAD_BATCH]
+            ops.gemm_wgrad_f32_batch([op for _, op in part],
+                                     main_grads=[weights[i].main_grad for i, _ in part])
+        for j in range(0, len(to_grad), _WGRAD_BATCH):
+            part = to_grad[j:j + _WGRAD_BATCH]
+            for (i, _), dw in zip(part, ops.gemm_wgrad_batch([op for _, op in part])):
+                grads[i] = dw if dw.dtype == weights[i].dtype else dw.to(weights[i].dtype)
         return (dx, *grads)
 
 
