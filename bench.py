@@ -585,7 +585,88 @@ def time_next_rows(o, bufs, stream, warmup, rounds):
         "what": "the same %d-layer step with power-of-two scales (s = 2^E, "
                 "the smallest E with 448*2^E >= amax) applied by the tensor "
                 "cores' UE8M0 block scaling; timed after the step" % LAYERS}
+    out["configs"] = time_configs(o, bufs, stream)
     return out
+
+
+def time_configs(o, bufs, stream, rounds=5):
+    """The single-linear workloads of the parity configurations, one kernel
+    at a time, each launch timed by CUDA events after an L2 flush (256 MB
+    written): the QKV fprop at 8192 tokens, the MLP fprop (gate/up, down) and
+    the MLP backward (dgrad and wgrad of down and gate/up) at 16384 tokens,
+    with the quantisers of their inputs. Operands are the step's buffers
+    (codes quantised during the step) where the shapes match."""
+    import torch
+    dev = bufs[0].x.device
+    by = {b.kind: b for b in bufs}
+    flush = torch.empty((256 << 20) if dev.type == "cuda" else 1024, dtype=torch.uint8,
+                        device=dev)
+    cd = lambda a: (a + 127) // 128  # noqa: E731
+
+    def timed(fn):
+        with torch.cuda.stream(stream):
+            fn()
+            fn()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(rounds)]
+        with torch.cuda.stream(stream):
+            for e0, e1 in evs:
+                flush.zero_()
+                e0.record(stream)
+                fn()
+                e1.record(stream)
+        torch.cuda.synchronize()
+        o.fp8bw_check_device_error(stream)
+        return sum(e0.elapsed_time(e1) for e0, e1 in evs) / rounds
+
+    rows = {}
+
+    def gemm_row(name, m, n, k, fn):
+        ms = timed(fn)
+        rows[name] = {"achieved": 2 * m * n * k / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                      "us": ms * 1e3, "shape": [m, n, k]}
+
+    def quant_row(name, nbytes, fn):
+        ms = timed(fn)
+        rows[name] = {"achieved": nbytes / (ms * 1e-3) / 1e9, "unit": "GB/s",
+                      "us": ms * 1e3, "bytes": nbytes}
+
+    if "qkv" in by:
+        b, m = by["qkv"], TOKENS // 2
+        x = b.x[:m]
+        qx = torch.empty((m, b.k), dtype=torch.uint8, device=dev)
+        sx = torch.empty((cd(b.k), m), dtype=torch.float32, device=dev)
+        y = torch.empty((m, b.n), dtype=torch.bfloat16, device=dev)
+        quant_row("qkv_m8192_quant_x_rowwise", m * b.k * 2 + m * b.k + 4 * m * cd(b.k),
+                  lambda: o.fp8bw_quantize_rowwise(x, qx, sx, stream))
+        gemm_row("qkv_m8192_fprop", m, b.n, b.k,
+                 lambda: o.fp8bw_gemm_fprop(qx, sx, b.qw, b.sw, y, stream))
+    m = TOKENS
+    for kind in ("gate_up", "down"):
+        if kind not in by:
+            continue
+        b = by[kind]
+        xq = m * b.k * 2 + 2 * m * b.k + 4 * (m * cd(b.k) + cd(m) * b.k)
+        dyq = m * b.n * 2 + 2 * m * b.n + 4 * (m * cd(b.n) + cd(m) * b.n)
+        quant_row(kind + "_quant_x_rowcol", xq,
+                  lambda b=b: o.fp8bw_quantize_colwise(b.x, b.qx_t, b.sx_t, b.qx, b.sx, stream))
+        gemm_row(kind + "_fprop", m, b.n, b.k,
+                 lambda b=b: o.fp8bw_gemm_fprop(b.qx, b.sx, b.qw, b.sw, b.y, stream))
+        quant_row(kind + "_quant_dy_rowcol", dyq,
+                  lambda b=b: o.fp8bw_quantize_colwise(b.dy, b.qdy_t, b.sdy_t, b.qdy, b.sdy,
+                                                       stream))
+        gemm_row(kind + "_dgrad", m, b.k, b.n,
+                 lambda b=b: o.fp8bw_gemm_dgrad(b.qdy, b.sdy, b.qw_t, 1, b.sw, b.dx, stream))
+        gemm_row(kind + "_wgrad", b.n, b.k, m,
+                 lambda b=b: o.fp8bw_gemm_wgrad(b.qdy_t, b.sdy_t, b.qx_t, b.sx_t, b.dw,
+                                                stream))
+    del flush
+    return {"rows": rows,
+            "what": "the parity configurations' linears one kernel at a time, L2 "
+                    "flushed before each launch (QKV fprop at M=%d; MLP fprop and "
+                    "backward at M=%d); shape = [rows, cols, contraction]; timed "
+                    "after the step" % (TOKENS // 2, TOKENS)}
 
 
 class ClockSampler:
@@ -929,10 +1010,14 @@ def result_line(args, world, res):
                "sample": sample.describe(), "seconds": dt}
 
     if next_rows is not None:
-        for d in next_rows.values():
+        entries = list(next_rows.values())
+        entries += list(next_rows.get("configs", {}).get("rows", {}).values())
+        for d in entries:
             if d.get("unit") == "TFLOP/s":
                 d["frac_of_fp8_peak"] = d["achieved"] / fp8_sustained
                 d["frac_of_fp8_peak_burst"] = d["achieved"] / fp8_burst
+            elif d.get("unit") == "GB/s":
+                d["frac_of_hbm"] = d["achieved"] / peaks["hbm_gbs"]
     value = weak_scaling_value(world, flops, ms * 1e-3) / 1e12
     line = {
         "metric": METRIC,

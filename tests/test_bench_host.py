@@ -79,8 +79,8 @@ class _FakeLinear:
     def __init__(self, kind, k, n):
         import torch
         self.kind, self.k, self.n = kind, k, n
-        for attr in ("w", "qx", "sx", "qw", "sw", "qw_t", "qdy", "sdy", "qdy_t",
-                     "sdy_t", "qx_t", "sx_t", "y", "dx"):
+        for attr in ("x", "dy", "dw", "w", "qx", "sx", "qw", "sw", "qw_t", "qdy", "sdy",
+                     "qdy_t", "sdy_t", "qx_t", "sx_t", "y", "dx"):
             setattr(self, attr, torch.zeros(1))
 
     def weight_bytes(self):
@@ -107,7 +107,11 @@ def test_next_rows_host_logic_with_stubbed_device(monkeypatch):
     bufs = [_FakeLinear("gate_up", 128, 256), _FakeLinear("down", 256, 128)]
     out = bench.time_next_rows(lib, bufs, None, 3, 5)
     assert set(out) == {"wgrad_f32_accumulate", "gemm_fused_rowwise_quant",
-                        "gemm_fused_rowcol_quant", "pow2_step"}
+                        "gemm_fused_rowcol_quant", "pow2_step", "configs"}
+    # the MLP configurations' kernels, one at a time (no QKV linear here)
+    assert set(out["configs"]["rows"]) == {
+        k + "_" + r for k in ("gate_up", "down")
+        for r in ("quant_x_rowcol", "fprop", "quant_dy_rowcol", "dgrad", "wgrad")}
     assert "gate/up and down linears" in out["wgrad_f32_accumulate"]["what"]
     assert "gate/up and down linears" in out["gemm_fused_rowwise_quant"]["what"]
     assert "gate/up and down linears" in out["gemm_fused_rowcol_quant"]["what"]
@@ -118,9 +122,13 @@ def test_next_rows_host_logic_with_stubbed_device(monkeypatch):
     assert lib.calls["fp8bw_gemm_wgrad_f32_batch"] == 3 + 5
     # the power-of-two step: one batched wgrad per layer
     assert lib.calls["fp8bw_gemm_wgrad_batch"] == 3 * bench.LAYERS + 3 * bench.LAYERS
-    # fprop runs in the row-wise and the row + column comparison alike
-    assert 2 * lib.calls["fp8bw_gemm_fprop_quant"] == lib.calls["fp8bw_gemm_fprop"]
+    # fprop runs in the row-wise and the row + column comparison alike, and
+    # in the configurations' timing (2 warm-up + 5 timed calls per linear)
+    assert 2 * lib.calls["fp8bw_gemm_fprop_quant"] + 2 * (2 + 5) == \
+        lib.calls["fp8bw_gemm_fprop"]
     assert set(out["pow2_step"]["breakdown"]) == {
         "quant_weight_block", "quant_rowcol", "gemm_block_scaled",
         "gemm_vector_scaled"}
-    assert all(v["unit"] == "TFLOP/s" for k, v in out.items())
+    assert all(v["unit"] == "TFLOP/s" for k, v in out.items() if k != "configs")
+    assert all(r["unit"] == ("TFLOP/s" if k.endswith(("fprop", "dgrad", "wgrad")) else "GB/s")
+               for k, r in out["configs"]["rows"].items())
