@@ -51,4 +51,9 @@ def test_gpu_arm_line_one_layer():
     assert e["value"] > 0 and e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] > 0
     assert d["clocks"] is None or d["clocks"]["sm_mhz"] > 0
     assert set(d["next_rows"]) == {"wgrad_f32_accumulate", "gemm_fused_rowwise_quant",
-                                   "gemm_fused_rowcol_quant", "pow2_step"}
+                                   "gemm_fused_rowcol_quant", "pow2_step", "configs"}
+    rows = d["next_rows"]["configs"]["rows"]
+    assert set(rows) == {"qkv_m8192_quant_x_rowwise", "qkv_m8192_fprop"}
+    assert rows["qkv_m8192_fprop"]["shape"] == [8192, 4096, 2048]
+    assert all(r["achieved"] > 0 and ("frac_of_fp8_peak" in r or "frac_of_hbm" in r)
+               for r in rows.values())

@@ -11,7 +11,10 @@ Checks:
     of different shapes (ragged edges, tile counts that do not fill a wave,
     a job of one tile), for both scale forms;
   * that empty jobs (n or k zero) are skipped and an empty contraction writes
-    zeros (or leaves a main-grad unchanged).
+    zeros (or leaves a main-grad unchanged);
+  * the bench step's launch at full size: a layer's four linears at M =
+    16384, bit-equal to the single calls and within the bound of the oracle
+    on sampled points.
 """
 import numpy as np
 import pytest
@@ -119,3 +122,32 @@ def test_empty_jobs_and_empty_contraction():
     ops.fp8bw_check_device_error()
     assert not dw.float().abs().sum().item()
     assert np.all(g.cpu().numpy() == np.float32(0.5))
+
+
+def test_full_size_layer_batch():
+    """The bench step's launch: the four linears of a layer (QKV, O, gate/up,
+    down) at M = 16384 in one batched wgrad. Each dW equals the single-problem
+    wgrad bit for bit, and sampled points (>= 16 per 128x128 tile plus two
+    full rows and columns) are within the acceptance bound of the oracle."""
+    from helpers import sample_points
+    ops = _ops()
+    m = 16384
+    jobs, ins = [], []
+    for kind in ("qkv", "o", "gate_up", "down"):
+        k, n = S.LINEARS[kind]
+        dy = S.bf16_normal((m, n), 0, S.tensor_id(kind, "dy", 0), **S.DY_DIST)
+        x = S.bf16_normal((m, k), 0, S.tensor_id(kind, "x", 0), **S.X_DIST)
+        jobs.append(ops.quantize_colwise(bf16_np_to_torch(dy)) +
+                    ops.quantize_colwise(bf16_np_to_torch(x)))
+        ins.append((dy, x, n, k))
+    dws = ops.gemm_wgrad_batch(jobs)
+    singles = [ops.gemm_wgrad(*j) for j in jobs]
+    ops.fp8bw_check_device_error()
+    for (dy, x, n, k), dw, single in zip(ins, dws, singles):
+        assert _eq(dw, single), "batched dW %dx%d differs from the single call" % (n, k)
+        rq, rs = oracle.quantize_colwise(dy)
+        rqx, rsx = oracle.quantize_colwise(x)
+        pi, pj = sample_points(n, k)
+        acc, bound = oracle.gemm_wgrad_points(rq, rs, rqx, rsx, pi, pj)
+        assert_gemm_close(torch_bf16_to_np(dw)[pi, pj], acc, bound,
+                          "batched wgrad %dx%dx%d" % (m, n, k))
